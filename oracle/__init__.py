@@ -1,0 +1,236 @@
+"""Float64 CPU oracle for GQA over a KV cache.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` are the only
+callers. The CUDA path never imports this package and this package never
+imports the CUDA path; the two share no code.
+
+The arithmetic lives in ``gqa_ref.c`` (plain loops in double). This module
+only marshals numpy arrays into it, and adds the two pieces that are not
+arithmetic: the per-token KV-cache size formula and the KV append (a row
+copy).
+
+Page citations (title, section):
+  * KV bytes per token S_KV = 2 * L * K * d_k * bytes: "GQA 完全拆解"
+    (pinghaoyang.com.cn), sections 解码推理的内存账本 and 主流模型里的 GQA：
+    KV 缓存账本 (there the KV-head count is written G); the per-layer element
+    count 2 * K * d_k: "分組查詢注意力" (compassingai.com), section 關鍵引數.
+  * KV append: "分組查詢注意力", section 技術原理 (each new token writes K and
+    V of shape [batch, 1, K, d_k]); "GQA 完全拆解", section 解码推理的内存账本
+    (after step t the new K, V row is appended to the cache).
+
+Parity status: pinned (tests/test_oracle_pins.py); nothing here is "parity
+unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gqa_ref.c")
+_LIB = os.path.join(_HERE, "libgqa_oracle.so")
+
+F32, BF16, F64 = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        # -ffp-contract=off: no fused multiply-add, every step rounds as written
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def load_library(path: str):
+    """Load an oracle build from ``path`` (the tests use this to load mutants)."""
+    return _declare(ctypes.CDLL(path))
+
+
+def _get(lib=None):
+    global _lib
+    if lib is not None:
+        return lib
+    if _lib is None:
+        _lib = _declare(ctypes.CDLL(build()))
+    return _lib
+
+
+def _declare(lib):
+    P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+    lib.ref_decode.restype = I
+    lib.ref_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, D, I, P, I64, I]
+    lib.ref_prefill_causal.restype = I
+    lib.ref_prefill_causal.argtypes = [P, P, P, P, I, I, I, I, I, D, I, P, I64, I]
+    lib.ref_meanpool.restype = I
+    lib.ref_meanpool.argtypes = [P, P, I64, I, I, I64, I]
+    lib.ref_round_bf16.argtypes = [P, P, I64]
+    lib.ref_round_f32.argtypes = [P, P, I64]
+    return lib
+
+
+def _threads(nthreads: Optional[int]) -> int:
+    if nthreads:
+        return int(nthreads)
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.float64:
+        return F64
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    raise TypeError(f"unsupported dtype {a.dtype}: float64, float32 or uint16 (bfloat16 bits)")
+
+
+def _c(a: np.ndarray) -> np.ndarray:
+    return np.ascontiguousarray(a)
+
+
+# ---------------------------------------------------------------------------
+# sizes
+
+def kv_cache_bytes_per_token(layers: int, kv_heads: int, head_dim: int, bytes_per_elt: int) -> int:
+    """S_KV = 2 * L * K * d_k * bytes (the factor 2: one K row and one V row)."""
+    return 2 * layers * kv_heads * head_dim * bytes_per_elt
+
+
+def kv_cache_elements_per_layer_token(kv_heads: int, head_dim: int) -> int:
+    """2 * K * d_k elements per layer and token."""
+    return 2 * kv_heads * head_dim
+
+
+# ---------------------------------------------------------------------------
+# arithmetic (float64)
+
+def decode(q, k_cache, v_cache, seqlens, scale: float, sel=None, nthreads=None, lib=None) -> np.ndarray:
+    """q [B,H,d], caches [B,K,S_max,d], seqlens [B] -> float64 [B,H,d].
+
+    With ``sel`` (an int array of (b, h) pairs) only those rows are computed and
+    the result is [len(sel), d].
+    """
+    q, k_cache, v_cache = _c(q), _c(k_cache), _c(v_cache)
+    B, H, d = q.shape
+    Bk, K, S_max, dk = k_cache.shape
+    assert Bk == B and dk == d and v_cache.shape == k_cache.shape
+    dt = _dtype_code(q)
+    assert _dtype_code(k_cache) == dt and _dtype_code(v_cache) == dt
+    seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
+    assert seqlens.shape == (B,)
+    if sel is None:
+        out = np.empty((B, H, d), dtype=np.float64)
+        selp, nsel = None, 0
+    else:
+        sel = np.ascontiguousarray(sel, dtype=np.int32).reshape(-1, 2)
+        out = np.empty((sel.shape[0], d), dtype=np.float64)
+        selp, nsel = sel.ctypes.data, sel.shape[0]
+    rc = _get(lib).ref_decode(out.ctypes.data, q.ctypes.data, k_cache.ctypes.data, v_cache.ctypes.data,
+                              seqlens.ctypes.data, B, H, K, S_max, d, float(scale), dt, selp, nsel,
+                              _threads(nthreads))
+    if rc != 0:
+        raise ValueError("oracle: H must be a multiple of K")
+    return out
+
+
+def prefill_causal(q, k, v, scale: float, sel=None, nthreads=None, lib=None) -> np.ndarray:
+    """q [B,S,H,d], k/v [B,S,K,d] -> float64 [B,S,H,d]; row i sees keys j <= i.
+
+    With ``sel`` (an int array of (b, i, h) triples) only those rows are
+    computed and the result is [len(sel), d].
+    """
+    q, k, v = _c(q), _c(k), _c(v)
+    B, S, H, d = q.shape
+    assert k.shape[:2] == (B, S) and k.shape[3] == d and v.shape == k.shape
+    K = k.shape[2]
+    dt = _dtype_code(q)
+    if sel is None:
+        out = np.empty((B, S, H, d), dtype=np.float64)
+        selp, nsel = None, 0
+    else:
+        sel = np.ascontiguousarray(sel, dtype=np.int32).reshape(-1, 3)
+        out = np.empty((sel.shape[0], d), dtype=np.float64)
+        selp, nsel = sel.ctypes.data, sel.shape[0]
+    rc = _get(lib).ref_prefill_causal(out.ctypes.data, q.ctypes.data, k.ctypes.data, v.ctypes.data,
+                                      B, S, H, K, d, float(scale), dt, selp, nsel, _threads(nthreads))
+    if rc != 0:
+        raise ValueError("oracle: H must be a multiple of K")
+    return out
+
+
+def meanpool_kv(src, K: int, lib=None) -> np.ndarray:
+    """src [outer, H, inner] -> float64 [outer, K, inner], mean over each group's H/K heads."""
+    src = _c(src)
+    outer, H, inner = src.shape
+    out = np.empty((outer, K, inner), dtype=np.float64)
+    rc = _get(lib).ref_meanpool(out.ctypes.data, src.ctypes.data, outer, H, K, inner, _dtype_code(src))
+    if rc != 0:
+        raise ValueError("oracle: H must be a multiple of K")
+    return out
+
+
+def round_to(x: np.ndarray, like_dtype) -> np.ndarray:
+    """Round float64 values to float32 or bfloat16 bits (uint16), nearest-even."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    if np.dtype(like_dtype) == np.float32:
+        out = np.empty(x.shape, dtype=np.float32)
+        _get().ref_round_f32(x.ctypes.data, out.ctypes.data, x.size)
+        return out
+    if np.dtype(like_dtype) == np.uint16:
+        out = np.empty(x.shape, dtype=np.uint16)
+        _get().ref_round_bf16(x.ctypes.data, out.ctypes.data, x.size)
+        return out
+    if np.dtype(like_dtype) == np.float64:
+        return x.copy()
+    raise TypeError(like_dtype)
+
+
+def widen(a: np.ndarray) -> np.ndarray:
+    """Stored values (float32, float64 or bfloat16 bits) as float64."""
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# KV append (a row copy)
+
+def kv_append(k_cache, v_cache, k_new, v_new, pos):
+    """Return copies of the caches with row pos[b] of every (b, g) set to the new token.
+
+    Positions outside [0, S_max) leave the cache untouched (the CUDA path
+    reports them as a device error instead of writing).
+    """
+    kc, vc = np.array(k_cache, copy=True), np.array(v_cache, copy=True)
+    B, K, S_max, _ = kc.shape
+    for b in range(B):
+        p = int(pos[b])
+        if 0 <= p < S_max:
+            kc[b, :, p, :] = k_new[b]
+            vc[b, :, p, :] = v_new[b]
+    return kc, vc
+
+
+def prefill_cache_write(k, v, S_max: int, k_cache=None, v_cache=None):
+    """k/v [B,S,K,d] -> caches [B,K,S_max,d] with rows 0..S-1 filled (others kept)."""
+    B, S, K, d = k.shape
+    if k_cache is None:
+        k_cache = np.zeros((B, K, S_max, d), dtype=k.dtype)
+        v_cache = np.zeros((B, K, S_max, d), dtype=v.dtype)
+    kc, vc = np.array(k_cache, copy=True), np.array(v_cache, copy=True)
+    kc[:, :, :S, :] = np.transpose(k, (0, 2, 1, 3))
+    vc[:, :, :S, :] = np.transpose(v, (0, 2, 1, 3))
+    return kc, vc

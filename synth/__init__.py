@@ -1,0 +1,202 @@
+"""Seeded synthetic inputs (numbers only; none of the attention arithmetic).
+
+Both the CUDA path and the float64 oracle are fed from here, so that they see
+identical input bytes while sharing no code. The generator is defined in
+``gen.c`` (splitmix64 counter stream, Box-Muller normals). bfloat16 data is
+held on the host as ``numpy.uint16`` bit patterns.
+
+The workloads are the Llama-shaped decode and prefill problems of the GQA
+pages: Llama-3-8B (32 query heads, 8 KV heads, head dim 128, "GQA 完全拆解",
+KV-cache ledger section), the 70B shape with 64 query heads over 8 KV heads
+("分組查詢注意力", key-parameters section), and 128K-token contexts (same
+ledger section). Every value is N(0, 1).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gen.c")
+_LIB = os.path.join(_HERE, "libsynth.so")
+
+F32, BF16, F64 = 0, 1, 2
+SEED_BASE = 0x6A510000
+STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_KNEW, STREAM_VNEW = 1, 2, 3, 4, 5, 6
+
+
+def build(force: bool = False) -> str:
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _get():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.synth_stream_key.restype = ctypes.c_uint64
+        lib.synth_stream_key.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        lib.synth_draw.restype = ctypes.c_uint64
+        lib.synth_draw.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        lib.synth_normal.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64,
+                                     ctypes.c_uint64, ctypes.c_int]
+        lib.synth_cache.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_int64,
+                                    ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+                                    ctypes.c_int]
+        lib.synth_uniform_int.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int64,
+                                          ctypes.c_int32, ctypes.c_int32]
+        _lib = lib
+    return _lib
+
+
+def host_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+def _np_dtype(dtype: int):
+    return {F32: np.float32, BF16: np.uint16, F64: np.float64}[dtype]
+
+
+def stream_key(seed: int, stream: int) -> int:
+    return int(_get().synth_stream_key(seed, stream))
+
+
+def draw(key: int, i: int) -> int:
+    return int(_get().synth_draw(key, i))
+
+
+def normal(shape, dtype: int, seed: int, stream: int, start: int = 0) -> np.ndarray:
+    out = np.empty(shape, dtype=_np_dtype(dtype))
+    if out.size:
+        _get().synth_normal(out.ctypes.data, dtype, stream_key(seed, stream), start, out.size, host_threads())
+    return out
+
+
+def cache(units: int, S_max: int, d: int, dtype: int, seed: int, stream: int,
+          lens: Optional[np.ndarray] = None, units_per_len: int = 1) -> np.ndarray:
+    """[units, S_max, d] cache; rows at or past lens[u // units_per_len] are quiet NaN."""
+    out = np.empty((units, S_max, d), dtype=_np_dtype(dtype))
+    lp = None
+    if lens is not None:
+        lens = np.ascontiguousarray(lens, dtype=np.int32)
+        lp = lens.ctypes.data
+    if out.size:
+        _get().synth_cache(out.ctypes.data, dtype, stream_key(seed, stream), units, S_max, d, lp,
+                           units_per_len, host_threads())
+    return out
+
+
+def uniform_int(n: int, lo: int, hi: int, seed: int, stream: int) -> np.ndarray:
+    out = np.empty(n, dtype=np.int32)
+    if n:
+        _get().synth_uniform_int(out.ctypes.data, stream_key(seed, stream), n, lo, hi)
+    return out
+
+
+# --------------------------------------------------------------------------
+# workloads
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeShape:
+    name: str
+    B: int
+    H: int
+    K: int
+    d: int
+    S_max: int
+    dtype: int
+    seed: int
+    lens: tuple = ()          # () -> every sequence has length S_max
+    len_range: tuple = ()     # (lo, hi) -> uniform integers drawn from the seed
+    append: bool = False      # one kv_append of the last token per step
+
+    @property
+    def G(self) -> int:
+        return self.H // self.K
+
+    @property
+    def elt(self) -> int:
+        return 4 if self.dtype == F32 else 2
+
+
+@dataclasses.dataclass(frozen=True)
+class PrefillShape:
+    name: str
+    B: int
+    S: int
+    H: int
+    K: int
+    d: int
+    dtype: int
+    seed: int
+
+
+DECODE_WORKLOADS = {
+    "tiny_decode_b1_h8_k2_d64_s128_f32": DecodeShape(
+        "tiny_decode_b1_h8_k2_d64_s128_f32", 1, 8, 2, 64, 128, F32, SEED_BASE + 0),
+    "llama3_8b_decode_b8_h32_k8_d128_s8192": DecodeShape(
+        "llama3_8b_decode_b8_h32_k8_d128_s8192", 8, 32, 8, 128, 8192, BF16, SEED_BASE + 1, append=True),
+    "ragged_70b_decode_b32_h64_k8_d128_s1k_16k": DecodeShape(
+        "ragged_70b_decode_b32_h64_k8_d128_s1k_16k", 32, 64, 8, 128, 16384, BF16, SEED_BASE + 2,
+        len_range=(1024, 16384)),
+    "long_ctx_gqa_b1_h64_k8_d128_s131072": DecodeShape(
+        "long_ctx_gqa_b1_h64_k8_d128_s131072", 1, 64, 8, 128, 131072, BF16, SEED_BASE + 3),
+    "long_ctx_mqa_b1_h64_k1_d128_s131072": DecodeShape(
+        "long_ctx_mqa_b1_h64_k1_d128_s131072", 1, 64, 1, 128, 131072, BF16, SEED_BASE + 3),
+}
+
+PREFILL_WORKLOADS = {
+    "causal_prefill_b4_s4096_h32_k8_d128": PrefillShape(
+        "causal_prefill_b4_s4096_h32_k8_d128", 4, 4096, 32, 8, 128, BF16, SEED_BASE + 4),
+}
+
+
+def seqlens_for(w: DecodeShape) -> np.ndarray:
+    if w.lens:
+        return np.asarray(w.lens, dtype=np.int32)
+    if w.len_range:
+        return uniform_int(w.B, w.len_range[0], w.len_range[1], w.seed, STREAM_LENS)
+    return np.full(w.B, w.S_max, dtype=np.int32)
+
+
+def decode_inputs(w: DecodeShape) -> dict:
+    """q [B,H,d], k/v cache [B,K,S_max,d] (NaN past each length), seqlens [B];
+    with ``append``: k_new/v_new [B,K,d] and pos [B] = seqlens - 1."""
+    lens = seqlens_for(w)
+    out = {
+        "q": normal((w.B, w.H, w.d), w.dtype, w.seed, STREAM_Q),
+        "k_cache": cache(w.B * w.K, w.S_max, w.d, w.dtype, w.seed, STREAM_K, lens, w.K).reshape(
+            w.B, w.K, w.S_max, w.d),
+        "v_cache": cache(w.B * w.K, w.S_max, w.d, w.dtype, w.seed, STREAM_V, lens, w.K).reshape(
+            w.B, w.K, w.S_max, w.d),
+        "seqlens": lens,
+    }
+    if w.append:
+        out["k_new"] = normal((w.B, w.K, w.d), w.dtype, w.seed, STREAM_KNEW)
+        out["v_new"] = normal((w.B, w.K, w.d), w.dtype, w.seed, STREAM_VNEW)
+        out["pos"] = (lens - 1).astype(np.int32)
+    return out
+
+
+def prefill_inputs(w: PrefillShape) -> dict:
+    """q [B,S,H,d], k/v [B,S,K,d]."""
+    return {
+        "q": normal((w.B, w.S, w.H, w.d), w.dtype, w.seed, STREAM_Q),
+        "k": normal((w.B, w.S, w.K, w.d), w.dtype, w.seed, STREAM_K),
+        "v": normal((w.B, w.S, w.K, w.d), w.dtype, w.seed, STREAM_V),
+    }

@@ -1,0 +1,47 @@
+"""The seeded input generator: deterministic, sliceable, N(0, 1), NaN past each length."""
+import numpy as np
+
+import synth
+
+
+def test_splitmix64_reference_values():
+    # splitmix64 seeded with 0: the published first outputs of the generator
+    assert synth.draw(0, 0) == 0xE220A8397B1DCDAF
+    assert synth.draw(0, 1) == 0x6E789E6AA1B965F4
+    assert synth.draw(0, 2) == 0x06C45D188009454F
+
+
+def test_normals_are_standard_and_sliceable():
+    x = synth.normal((1 << 18,), synth.F64, 7, 1)
+    assert abs(x.mean()) < 0.01 and abs(x.std() - 1) < 0.01
+    key = synth.stream_key(7, 1)
+    part = np.empty(1001, np.float64)
+    synth._get().synth_normal(part.ctypes.data, synth.F64, key, 777, part.size, 3)
+    assert np.array_equal(part, x[777:1778])
+
+
+def test_dtypes_round_the_same_draws():
+    x64 = synth.normal((4096,), synth.F64, 3, 2)
+    x32 = synth.normal((4096,), synth.F32, 3, 2)
+    xb = synth.normal((4096,), synth.BF16, 3, 2)
+    assert np.array_equal(x32, x64.astype(np.float32))
+    widened = (xb.astype(np.uint32) << 16).view(np.float32)
+    assert np.max(np.abs(widened - x32) / np.maximum(np.abs(x32), 1e-30)) <= 2.0**-8
+
+
+def test_cache_rows_past_length_are_nan():
+    lens = np.array([3, 0, 5], np.int32)
+    c = synth.cache(6, 5, 4, synth.F32, 9, 2, lens, 2)
+    full = synth.normal((6, 5, 4), synth.F32, 9, 2)
+    for u in range(6):
+        n = lens[u // 2]
+        assert np.array_equal(c[u, :n], full[u, :n])
+        assert np.isnan(c[u, n:]).all()
+
+
+def test_uniform_int_range_and_workload_lengths():
+    v = synth.uniform_int(10000, 1024, 16384, 5, 4)
+    assert v.min() >= 1024 and v.max() <= 16384
+    w = synth.DECODE_WORKLOADS["ragged_70b_decode_b32_h64_k8_d128_s1k_16k"]
+    lens = synth.seqlens_for(w)
+    assert lens.shape == (32,) and lens.min() >= 1024 and lens.max() <= 16384
