@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark: GQA decode effective HBM GB/s on B200 (plus prefill TFLOP/s).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one token's attention work for a Llama-3-8B-shaped model: for each
+of its 32 layers, one gqa_kv_append of the new token's K/V rows and one
+gqa_decode of the 8 x 32 query heads over the 8 x 8 KV heads at context 8192
+(bf16, head dim 128). Every layer has its own 256 MiB cache pair, so a step
+streams 8 GiB, far more than the 126 MB L2; no flush is needed.
+
+value = KV bytes that decode must read (each cached row once) / step time.
+N > 1 runs independent replicas (one per GPU, no data-path collective): value
+is the sum over ranks of the bytes processed divided by the slowest rank's
+time.
+
+--impl reference times the float64 CPU oracle on the host cores instead (the
+reference arm), one (batch, KV head) unit of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "llama3_8b_decode_b8_h32_k8_d128_s8192"
+LAYERS = 32
+METRIC = "GQA decode effective HBM GB/s"
+UNIT = "GB/s"
+
+
+# ---------------------------------------------------------------------------
+# multi-rank plumbing (also exercised on CPU with gloo by the tests)
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def aggregate(local_ms: float, local_bytes: float, group=None):
+    """(max time over ranks in ms, total bytes over ranks) via all_reduce."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return local_ms, local_bytes
+    backend = dist.get_backend(group)
+    dev = "cuda" if backend == "nccl" else "cpu"
+    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
+    b = torch.tensor([local_bytes], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM, group=group)
+    return float(t.item()), float(b.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML polling thread)
+
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, interval_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.index, self.interval = index, interval_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - no NVML
+            self._nv, self.error = None, str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self._nv:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self._nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        reasons = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": reasons}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def profiled_traffic(name: str, source_files):
+    """ncu DRAM bytes per launch from profiles/<name>.json, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", f"{name}.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for s in source_files:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    if rec.get("source_sha256") != h.hexdigest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+def bench_ours(args, rank, world, local):
+    import torch
+
+    from kv_cache_02_b200 import gqa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.DECODE_WORKLOADS[WORKLOAD]
+    inp = synth.decode_inputs(w)
+    B, H, K, d, S = w.B, w.H, w.K, w.d, w.S_max
+    scale = 1.0 / np.sqrt(d)
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).to(dev)
+
+    kc1, vc1 = to_dev(inp["k_cache"]), to_dev(inp["v_cache"])
+    kc = torch.empty((LAYERS, B, K, S, d), dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    for layer in range(LAYERS):
+        kc[layer].copy_(kc1)
+        vc[layer].copy_(vc1)
+    del kc1, vc1
+    q = to_dev(inp["q"]).unsqueeze(0).repeat(LAYERS, 1, 1, 1).contiguous()
+    k_new = to_dev(inp["k_new"]).unsqueeze(0).repeat(LAYERS, 1, 1, 1).contiguous()
+    v_new = to_dev(inp["v_new"]).unsqueeze(0).repeat(LAYERS, 1, 1, 1).contiguous()
+    pos = to_dev(inp["pos"])
+    seqlens = to_dev(inp["seqlens"])
+    out = torch.empty_like(q)
+    ws_bytes = gqa.gqa_decode_workspace_bytes(B, H, K, S, d, 0)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    launches_per_layer = 1 + (2 if ws_bytes > 0 else 1)
+    kv_bytes_layer = 2 * B * K * S * d * 2  # K and V, every row once
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        for layer in range(LAYERS):
+            gqa.gqa_kv_append(kc[layer], vc[layer], k_new[layer], v_new[layer], pos)
+            if ev is not None:
+                ev[layer][0].record(stream)
+            gqa.gqa_decode(out[layer], q[layer], kc[layer], vc[layer], seqlens, scale, 0, ws)
+            if ev is not None:
+                ev[layer][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = gqa.gqa_get_last_error()
+    if status != (0, 0):
+        raise RuntimeError(f"device error during warm-up: {status}")
+
+    import torch.distributed as dist
+
+    dec_events = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(LAYERS)]
+                  for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for s in range(args.steps):
+            step(dec_events[s])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    local_ms = t0.elapsed_time(t1)
+    dec_ms = [dec_events[s][l][0].elapsed_time(dec_events[s][l][1]) for s in range(args.steps) for l in range(LAYERS)]
+    status = gqa.gqa_get_last_error()
+    if status != (0, 0):
+        raise RuntimeError(f"device error in the timed region: {status}")
+
+    max_ms, total_bytes = aggregate(local_ms, kv_bytes_layer * LAYERS * args.steps)
+    value = total_bytes / (max_ms * 1e-3) / 1e9
+    ms_per_step = max_ms / args.steps
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    q_h = q.cpu().pin_memory()
+    kn_h, vn_h = k_new.cpu().pin_memory(), v_new.cpu().pin_memory()
+    pos_h = pos.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        k_new.copy_(kn_h, non_blocking=True)
+        v_new.copy_(vn_h, non_blocking=True)
+        pos.copy_(pos_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms_local = e0.elapsed_time(e1)
+    e2e_max_ms, e2e_bytes = aggregate(e2e_ms_local, kv_bytes_layer * LAYERS * e2e_steps)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, kn_h, vn_h, pos_h))
+    d2h = out_h.numel() * out_h.element_size()
+
+    peaks, peak_src = measured_peaks()
+    dec_avg_ms = statistics.fmean(dec_ms)
+    achieved = kv_bytes_layer / (dec_avg_ms * 1e-3) / 1e9
+    traffic = profiled_traffic("decode_bf16_llama3_8b_traffic",
+                               ["kv_cache_02_b200/csrc/decode.cuh", "kv_cache_02_b200/csrc/common.cuh"])
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "H": H, "K": K, "d": d, "context": S,
+                   "layers_per_step": LAYERS, "kv_append_per_layer": True,
+                   "l2": "inputs larger than L2: each step streams 32 distinct 256 MiB cache pairs (8 GiB)",
+                   "parallelism": f"replicas x{world}", "num_splits": "auto"},
+        "roofline": {"bound": "hbm", "kernel": "gqa_decode (decode_bf16_kernel + decode_combine_kernel)",
+                     "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "peak_source": peak_src,
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": traffic, "algorithmic_bytes_per_launch": kv_bytes_layer,
+                     "avg_launch_ms": round(dec_avg_ms, 5)},
+        "e2e": {"value": round(e2e_bytes / (e2e_max_ms * 1e-3) / 1e9, 1), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "pinned-host q, k_new, v_new, pos copied in and out copied back every step; "
+                        "the KV cache is device-resident state"},
+        "gpu_launches": launches_per_layer * LAYERS * args.steps,
+        "clocks": clocks.summary(),
+    }
+    return result, dict(inp=inp, scale=scale, kv_bytes_layer=kv_bytes_layer)
+
+
+def extra_measurements(args):
+    """Other workloads, rank 0 at N = 1: decode configs and the causal prefill."""
+    import torch
+
+    from kv_cache_02_b200 import gqa
+
+    peaks, _ = measured_peaks()
+    res = {}
+    for name in ["ragged_70b_decode_b32_h64_k8_d128_s1k_16k", "long_ctx_gqa_b1_h64_k8_d128_s131072",
+                 "long_ctx_mqa_b1_h64_k1_d128_s131072"]:
+        w = synth.DECODE_WORKLOADS[name]
+        inp = synth.decode_inputs(w)
+
+        def to_dev(a):
+            t = torch.from_numpy(np.ascontiguousarray(a))
+            return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).cuda()
+
+        q, kc, vc, lens = to_dev(inp["q"]), to_dev(inp["k_cache"]), to_dev(inp["v_cache"]), to_dev(inp["seqlens"])
+        out = torch.empty_like(q)
+        wsb = gqa.gqa_decode_workspace_bytes(w.B, w.H, w.K, w.S_max, w.d, 0)
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+        flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        kv_bytes = int(inp["seqlens"].astype(np.int64).sum()) * w.K * w.d * 2 * 2
+        times = []
+        for it in range(args.warmup + 20):
+            flush.zero_()  # evict the previous iteration's cache rows from L2
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            gqa.gqa_decode(out, q, kc, vc, lens, 1.0 / np.sqrt(w.d), 0, ws)
+            b.record()
+            torch.cuda.synchronize()
+            if it >= args.warmup:
+                times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        gbs = kv_bytes / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 5), "kv_bytes": kv_bytes, "GB/s": round(gbs, 1),
+                     "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "l2": "flushed (512 MiB write)"}
+        del q, kc, vc, out, ws, flush
+        torch.cuda.empty_cache()
+    if gqa.gqa_get_last_error() != (0, 0):
+        raise RuntimeError("device error in extra measurements")
+    return res
+
+
+def cpu_baseline(inp, scale, kv_bytes_layer):
+    """The oracle as it stands, on all host cores, over one full layer of the workload."""
+    import oracle
+
+    threads = synth.host_threads()
+    t = time.perf_counter()
+    oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], scale, nthreads=threads)
+    dt = time.perf_counter() - t
+    return {"value": round(kv_bytes_layer / dt / 1e9, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"one layer of the step (all 8 x 32 heads over 8192 keys), {dt:.2f} s"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+
+def bench_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+
+    w = synth.DECODE_WORKLOADS[WORKLOAD]
+    inp = synth.decode_inputs(w)
+    threads = synth.host_threads()
+    scale = 1.0 / np.sqrt(w.d)
+    # one (batch, KV head) unit per step: all G query heads of that group over the full context
+    sel_all = [np.array([[b, g * w.G + j] for j in range(w.G)], np.int32) for b in range(w.B) for g in range(w.K)]
+    unit_bytes = 2 * w.S_max * w.d * 2
+    for i in range(args.warmup):
+        oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], scale, sel=sel_all[i % len(sel_all)],
+                      nthreads=threads)
+    t = time.perf_counter()
+    for i in range(args.steps):
+        oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], scale, sel=sel_all[i % len(sel_all)],
+                      nthreads=threads)
+    dt = time.perf_counter() - t
+    value = unit_bytes * args.steps / dt / 1e9
+    sample = "one (batch, KV head) unit per step: 4 query heads over 8192 keys"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "K": w.K, "d": w.d, "context": w.S_max,
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads and the CPU baseline")
+    ap.add_argument("--layers", type=int, default=32,
+                    help="layers per step (32 for the model; fewer only for small profiling captures)")
+    args = ap.parse_args()
+    global LAYERS
+    LAYERS = args.layers
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_env()
+
+    if args.impl == "reference":
+        res = bench_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        res, ctx = bench_ours(args, rank, world, local)
+        if rank == 0:
+            if world == 1 and not args.no_extra:
+                res["cpu_baseline"] = cpu_baseline(ctx["inp"], ctx["scale"], ctx["kv_bytes_layer"])
+                res["extra"] = extra_measurements(args)
+            elif world == 1:
+                res["cpu_baseline"] = None
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * gqa.h - grouped-query attention (GQA) over a KV cache, for NVIDIA B200
+ * (sm_100a). C ABI of libgqa.so.
+ *
+ * Notation: B batch, H query heads, K KV heads, G = H / K query heads per
+ * group, d head dimension, S_max cache capacity in tokens, len_b = seqlens[b].
+ * Query head h reads KV head h / G (contiguous grouping): "分組查詢注意力"
+ * (compassingai.com), section 技術原理, reshapes Q [b,s,H,d_k] into
+ * [b,s,K,H/K,d_k]; "GQA 完全拆解" (pinghaoyang.com.cn), section "GQA：插值在
+ * MHA 与 MQA 之间的分组共享", gives group g the consecutive heads
+ * (g-1)h/G+1 .. gh/G.
+ *
+ * Cache layout: [B, K, S_max, d], row-major. Each (b, g) slab is contiguous,
+ * rows are d elements ("GQA 完全拆解", section 工程实现, organises the cache
+ * as layer x KV head x position; "LLaMa3与DeepSeek采用的GQA技术" (CSDN),
+ * section 3, keeps each group's KV contiguous).
+ *
+ * Conventions shared by every call:
+ *  - All pointers are DEVICE pointers unless stated otherwise. The caller
+ *    owns every buffer; the library allocates no device memory.
+ *  - Every tensor is contiguous and its base address is 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream). The return value reports host-side validation and the
+ *    kernel launch only. Problems found on the device (an append position
+ *    outside the cache, a length outside [0, S_max], a bounded pipeline wait
+ *    that expired) never trap: they set bits of a per-device error word that
+ *    gqa_get_last_error() reads and clears.
+ *  - dtype is the storage type of every floating-point tensor of the call;
+ *    outputs use the same type. Arithmetic: float32 accumulation.
+ *  - Supported head dimensions: 64 and 128. H must be a multiple of K.
+ */
+#ifndef GQA_H_
+#define GQA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GQA_API __attribute__((visibility("default")))
+#else
+#define GQA_API
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* gqa_stream_t;
+
+typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
+
+typedef enum {
+  GQA_OK = 0,
+  GQA_ERR_INVALID_ARG = -1, /* NULL pointer, negative size, bad dtype, workspace too small */
+  GQA_ERR_SHAPE = -2,       /* H % K != 0, d not in {64, 128}, sizes beyond int32 indexing */
+  GQA_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
+  GQA_ERR_CUDA = -4,        /* a CUDA call or kernel launch failed */
+  GQA_ERR_DEVICE = -5,      /* the device error word was set (see GQA_DEVERR_*) */
+  GQA_ERR_UNSUPPORTED = -6  /* valid request that this build does not implement (e.g. f32 prefill) */
+} gqa_status;
+
+/* Bits of the device error word. */
+#define GQA_DEVERR_APPEND_POS 0x1u /* gqa_kv_append: pos[b] outside [0, S_max); row not written */
+#define GQA_DEVERR_SEQLEN 0x2u     /* gqa_decode: seqlens[b] outside [0, S_max]; out[b] set to zero */
+#define GQA_DEVERR_TIMEOUT 0x4u    /* a bounded wait in a pipelined kernel expired; output invalid */
+
+/*
+ * gqa_kv_append - write one new token's K and V rows into the cache.
+ *
+ * Defined by "分組查詢注意力", section 技術原理 (each new token writes K and V
+ * of shape [batch, 1, K, d_k], not [batch, 1, H, d_k]) and "GQA 完全拆解",
+ * section 解码推理的内存账本 (after decode step t the new K, V row is appended).
+ *
+ *   k_cache[b, g, pos[b], :] = k_new[b, g, :]   for every b < B, g < K
+ *   v_cache[b, g, pos[b], :] = v_new[b, g, :]
+ *
+ * k_cache, v_cache : [B, K, S_max, d], written in place (only those rows).
+ * k_new, v_new     : [B, K, d].
+ * pos              : [B] int32, device. pos[b] is the length of sequence b
+ *                    before the append; the decode that follows uses
+ *                    seqlens[b] = pos[b] + 1 so the new token sees itself.
+ * A position outside [0, S_max) is not written and sets GQA_DEVERR_APPEND_POS.
+ */
+GQA_API int gqa_kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* pos, int B,
+                  int K, int S_max, int d, gqa_dtype dtype, gqa_stream_t stream);
+
+/*
+ * gqa_decode_workspace_bytes - device workspace gqa_decode needs for the
+ * split-KV partial results of this shape (0 when no split is needed).
+ * num_splits as for gqa_decode (0 = automatic). Returns 0 for invalid shapes.
+ */
+GQA_API size_t gqa_decode_workspace_bytes(int B, int H, int K, int S_max, int d, int num_splits);
+
+/*
+ * gqa_decode - one decode step: every query head attends to its group's
+ * cached keys and values.
+ *
+ * Defined by "GQA 完全拆解", section 解码推理的内存账本 (at step t the new Q_t
+ * attends to all cached K_1..t, V_1..t) and section "GQA：插值在 MHA 与 MQA
+ * 之间的分组共享" (head i of group g uses the group's shared K_g, V_g);
+ * "LLaMa3与DeepSeek采用的GQA技术", section 2 (scores = q k^T / sqrt(d_k),
+ * softmax, weighted sum of V):
+ *
+ *   out[b, h, :] = sum_{t < len_b} softmax_t(scale * q[b,h,:] . k[b,g,t,:]) v[b,g,t,:],
+ *   g = h / (H / K)
+ *
+ * out       : [B, H, d], written.
+ * q         : [B, H, d].
+ * k_cache   : [B, K, S_max, d]; v_cache likewise. Rows t >= len_b are never
+ *             read into the result (their contents do not matter).
+ * seqlens   : [B] int32, device. len_b == 0 gives out[b] = 0. A value outside
+ *             [0, S_max] sets GQA_DEVERR_SEQLEN and gives out[b] = 0.
+ * scale     : the score scale, normally 1/sqrt(d).
+ * num_splits: how many key-axis partitions per (b, g) (split-KV with a
+ *             log-sum-exp combine); 0 picks one from the shape and the GPU.
+ * workspace : device scratch of at least gqa_decode_workspace_bytes(...)
+ *             bytes for the same shape and num_splits; may be NULL when that
+ *             size is 0. Its contents need no initialisation. Two calls that
+ *             share a workspace must not overlap on the GPU.
+ */
+GQA_API int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
+               int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+               gqa_dtype dtype, gqa_stream_t stream);
+
+/*
+ * gqa_prefill_causal - causal self-attention over a whole prompt, and the
+ * write of its keys and values into the cache.
+ *
+ * "GQA 完全拆解", section 解码推理的内存账本 (prefill processes the whole
+ * sequence in parallel) and section 质量与速度的实测权衡 (prefill is compute
+ * bound and writes the KV once). Causal mask: query row i sees keys j <= i.
+ *
+ *   out[b, i, h, :] = sum_{j <= i} softmax_j(scale * q[b,i,h,:] . k[b,j,g,:]) v[b,j,g,:]
+ *
+ * out        : [B, S, H, d], written.
+ * q          : [B, S, H, d].
+ * k, v       : [B, S, K, d].
+ * k_cache,
+ * v_cache    : [B, K, S_max, d] or both NULL. When given, rows 0..S-1 of
+ *              every (b, g) are set to k[b, :, g, :] / v[b, :, g, :]; other
+ *              rows are left as they are. Requires S <= S_max.
+ * dtype      : GQA_BF16 only (GQA_F32 returns GQA_ERR_UNSUPPORTED).
+ */
+GQA_API int gqa_prefill_causal(void* out, const void* q, const void* k, const void* v, void* k_cache, void* v_cache, int B,
+                       int S, int H, int K, int S_max, int d, float scale, gqa_dtype dtype, gqa_stream_t stream);
+
+/*
+ * gqa_meanpool_kv - MHA -> GQA conversion by mean pooling of heads.
+ *
+ * "分組查詢注意力", section 模型轉換與 Uptraining, and "GQA 完全拆解", section
+ * Uptraining: the new K (and V) head of group g is the arithmetic mean of the
+ * group's H/K original heads; Q is unchanged.
+ *
+ *   dst[o, g, i] = (1 / G) * sum_{r < G} src[o, g*G + r, i]
+ *
+ * src : [outer, H, inner]; dst : [outer, K, inner].
+ * Projection weights [H, d_k, d_model] use outer = 1, inner = d_k * d_model;
+ * per-head tensors [B, H, S, d] use outer = B, inner = S * d.
+ * The sum runs in float64 in ascending head order and is rounded once
+ * (nearest-even) to dtype, so the result is the correctly rounded mean
+ * whenever the float64 sum is exact (always for bf16 inputs within the
+ * normal range and G <= 2^16).
+ */
+GQA_API int gqa_meanpool_kv(void* dst, const void* src, int64_t outer, int H, int K, int64_t inner, gqa_dtype dtype,
+                    gqa_stream_t stream);
+
+/*
+ * gqa_get_last_error - synchronise `stream`, then read and clear the device
+ * error word of the current device. Returns GQA_OK when it was clear,
+ * GQA_ERR_DEVICE when any bit was set (bits stored to *bits if bits != NULL;
+ * bits is a HOST pointer), GQA_ERR_CUDA if the synchronisation failed.
+ */
+GQA_API int gqa_get_last_error(gqa_stream_t stream, uint32_t* bits);
+
+/* Human-readable name of a gqa_status value (static storage). */
+GQA_API const char* gqa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_H_ */

@@ -1,0 +1,330 @@
+// libgqa.so: the C ABI declared in include/gqa.h.
+//
+// Host side only validates arguments, plans the launch and encodes TMA
+// descriptors; every step of the computation runs in the kernels included
+// below. The library allocates no device memory: callers own all buffers,
+// including the decode workspace.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/gqa.h"
+#include "append_meanpool.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+using gqa::DecodeParams;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+int sm_count(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// cuTensorMapEncodeTiled from the driver, found through the runtime so the
+// library does not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over rows of `cols` elements, box = box_rows x 64 columns
+// (128 bytes), 128-byte swizzle. Rows past `rows` read as zero.
+bool encode_rows_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA; }
+
+// ----------------------------------------------------------------------------
+// decode launch plan
+
+struct DecodePlan {
+  int chunk = 0;    // keys per split (multiple of 64)
+  int nsplit = 1;   // splits per (b, g)
+  int hslices = 1;  // head slices per (b, g)
+  long long grid = 0;
+  size_t ws_bytes = 0;
+};
+
+bool valid_decode_shape(int B, int H, int K, int S_max, int d) {
+  if (B < 0 || H <= 0 || K <= 0 || S_max <= 0) return false;
+  if (H % K != 0) return false;
+  if (d != 64 && d != 128) return false;
+  if ((long long)B * K * S_max >= (1ll << 31)) return false;  // TMA row coordinate is int32
+  if ((long long)B * H >= (1ll << 31)) return false;
+  return true;
+}
+
+DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gqa_dtype dt, int sms) {
+  DecodePlan pl;
+  const int G = H / K;
+  const int heads_per_cta = dt == GQA_BF16 ? gqa::kDecHeadsPerCta : gqa::kDecF32HeadsPerCta;
+  pl.hslices = (G + heads_per_cta - 1) / heads_per_cta;
+  const long long units = (long long)B * K * pl.hslices;
+  const int max_splits = (S_max + 63) / 64;
+  int splits;
+  if (num_splits > 0) {
+    splits = std::min(num_splits, max_splits);
+  } else {
+    // about four waves of two CTAs per SM, never below 256 keys per split
+    const long long target = 8ll * sms;
+    splits = (int)std::max<long long>(1, (target + units - 1) / std::max<long long>(units, 1));
+    splits = std::min(splits, std::max(1, (S_max + 255) / 256));
+    splits = std::min(splits, max_splits);
+  }
+  int chunk = (S_max + splits - 1) / splits;
+  chunk = (chunk + 63) / 64 * 64;
+  pl.chunk = chunk;
+  pl.nsplit = (S_max + chunk - 1) / chunk;
+  pl.grid = (long long)B * K * pl.nsplit * pl.hslices;
+  if (pl.nsplit > 1) {
+    const size_t parts = (size_t)B * K * pl.nsplit * G;
+    pl.ws_bytes = parts * d * sizeof(float) + parts * sizeof(float2);
+  }
+  return pl;
+}
+
+template <int D>
+int launch_decode_bf16(const DecodePlan& pl, const DecodeParams& p, const void* kc, const void* vc, int B, int K,
+                       int S_max, cudaStream_t st) {
+  CUtensorMap tk, tv;
+  const uint64_t rows = (uint64_t)B * K * S_max;
+  if (!encode_rows_bf16(&tk, kc, rows, D, gqa::kDecBoxRows) || !encode_rows_bf16(&tv, vc, rows, D, gqa::kDecBoxRows))
+    return GQA_ERR_CUDA;
+  using C = gqa::DecCfg<D>;
+  static int configured[kMaxDevices] = {0};
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
+    if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      return GQA_ERR_CUDA;
+    configured[dev] = 1;
+  }
+  gqa::decode_bf16_kernel<D><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(tk, tv, p);
+  return launch_status();
+}
+
+template <int D>
+int launch_decode_f32(const DecodePlan& pl, const DecodeParams& p, const void* kc, const void* vc,
+                      cudaStream_t st) {
+  gqa::decode_f32_kernel<D><<<(unsigned)pl.grid, gqa::kDecF32Threads, 0, st>>>(
+      static_cast<const float*>(kc), static_cast<const float*>(vc), p);
+  return launch_status();
+}
+
+int grid_for(long long work_items, int threads, int sms) {
+  long long blocks = (work_items + threads - 1) / threads;
+  long long cap = (long long)sms * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return (int)blocks;
+}
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+
+extern "C" {
+
+const char* gqa_status_string(int status) {
+  switch (status) {
+    case GQA_OK: return "GQA_OK";
+    case GQA_ERR_INVALID_ARG: return "GQA_ERR_INVALID_ARG";
+    case GQA_ERR_SHAPE: return "GQA_ERR_SHAPE";
+    case GQA_ERR_ALIGN: return "GQA_ERR_ALIGN";
+    case GQA_ERR_CUDA: return "GQA_ERR_CUDA";
+    case GQA_ERR_DEVICE: return "GQA_ERR_DEVICE";
+    case GQA_ERR_UNSUPPORTED: return "GQA_ERR_UNSUPPORTED";
+    default: return "GQA_ERR_UNKNOWN";
+  }
+}
+
+int gqa_kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* pos, int B,
+                  int K, int S_max, int d, gqa_dtype dtype, gqa_stream_t stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (B < 0 || K <= 0 || S_max <= 0) return GQA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return GQA_ERR_SHAPE;
+  if (B == 0) return GQA_OK;
+  if (!k_cache || !v_cache || !k_new || !v_new || !pos) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new)) return GQA_ERR_ALIGN;
+  const int elt = dtype == GQA_F32 ? 4 : 2;
+  const int cpr = d * elt / 16;
+  const long long work = 2ll * B * K * cpr;
+  const int dev = current_device();
+  const int grid = grid_for(work, 256, sm_count(dev));
+  gqa::kv_append_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k_new),
+      static_cast<const uint4*>(v_new), pos, B, K, S_max, cpr);
+  return launch_status();
+}
+
+size_t gqa_decode_workspace_bytes(int B, int H, int K, int S_max, int d, int num_splits) {
+  if (!valid_decode_shape(B, H, K, S_max, d) || num_splits < 0) return 0;
+  const int dev = current_device();
+  // the plan does not depend on the dtype except through the head slicing,
+  // which does not change the workspace size; take the larger of the two
+  const DecodePlan a = plan_decode(B, H, K, S_max, d, num_splits, GQA_BF16, sm_count(dev));
+  const DecodePlan b = plan_decode(B, H, K, S_max, d, num_splits, GQA_F32, sm_count(dev));
+  return std::max(a.ws_bytes, b.ws_bytes);
+}
+
+int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
+               int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+               gqa_dtype dtype, gqa_stream_t stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (num_splits < 0 || B < 0 || H <= 0 || K <= 0 || S_max <= 0) return GQA_ERR_INVALID_ARG;
+  if (!valid_decode_shape(B, H, K, S_max, d)) return GQA_ERR_SHAPE;
+  if (B == 0) return GQA_OK;
+  if (!out || !q || !k_cache || !v_cache || !seqlens) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return GQA_ERR_ALIGN;
+  const int dev = current_device();
+  const DecodePlan pl = plan_decode(B, H, K, S_max, d, num_splits, dtype, sm_count(dev));
+  if (pl.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < pl.ws_bytes) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return GQA_ERR_ALIGN;
+  }
+  const int G = H / K;
+  DecodeParams p;
+  p.q = q;
+  p.out = out;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = pl.ws_bytes ? reinterpret_cast<float2*>(static_cast<char*>(workspace) +
+                                                    (size_t)B * K * pl.nsplit * G * d * sizeof(float))
+                        : nullptr;
+  p.seqlens = seqlens;
+  p.B = B;
+  p.H = H;
+  p.K = K;
+  p.S_max = S_max;
+  p.G = G;
+  p.hslices = pl.hslices;
+  p.chunk = pl.chunk;
+  p.nsplit = pl.nsplit;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = (cudaStream_t)stream;
+  int rc;
+  if (dtype == GQA_BF16)
+    rc = d == 128 ? launch_decode_bf16<128>(pl, p, k_cache, v_cache, B, K, S_max, st)
+                  : launch_decode_bf16<64>(pl, p, k_cache, v_cache, B, K, S_max, st);
+  else
+    rc = d == 128 ? launch_decode_f32<128>(pl, p, k_cache, v_cache, st)
+                  : launch_decode_f32<64>(pl, p, k_cache, v_cache, st);
+  if (rc != GQA_OK || pl.nsplit == 1) return rc;
+  if (dtype == GQA_BF16)
+    gqa::decode_combine_kernel<__nv_bfloat16><<<(unsigned)((long long)B * H), d, 0, st>>>(
+        static_cast<__nv_bfloat16*>(out), p.ws_o, p.ws_ml, seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, d);
+  else
+    gqa::decode_combine_kernel<float><<<(unsigned)((long long)B * H), d, 0, st>>>(
+        static_cast<float*>(out), p.ws_o, p.ws_ml, seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, d);
+  return launch_status();
+}
+
+int gqa_prefill_causal(void* out, const void* q, const void* k, const void* v, void* k_cache, void* v_cache, int B,
+                       int S, int H, int K, int S_max, int d, float scale, gqa_dtype dtype, gqa_stream_t stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (B < 0 || S < 0 || H <= 0 || K <= 0) return GQA_ERR_INVALID_ARG;
+  if (H % K != 0 || (d != 64 && d != 128)) return GQA_ERR_SHAPE;
+  if ((k_cache == nullptr) != (v_cache == nullptr)) return GQA_ERR_INVALID_ARG;
+  if (k_cache && S > S_max) return GQA_ERR_SHAPE;
+  if (B == 0 || S == 0) return GQA_OK;
+  if (!out || !q || !k || !v) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return GQA_ERR_ALIGN;
+  if (k_cache && (!aligned16(k_cache) || !aligned16(v_cache))) return GQA_ERR_ALIGN;
+  if (dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
+  return gqa::launch_prefill(out, q, k, v, k_cache, v_cache, B, S, H, K, S_max, d, scale, (cudaStream_t)stream,
+                             sm_count(current_device()));
+}
+
+int gqa_meanpool_kv(void* dst, const void* src, int64_t outer, int H, int K, int64_t inner, gqa_dtype dtype,
+                    gqa_stream_t stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (outer < 0 || inner < 0 || H <= 0 || K <= 0) return GQA_ERR_INVALID_ARG;
+  if (H % K != 0) return GQA_ERR_SHAPE;
+  if (outer == 0 || inner == 0) return GQA_OK;
+  if (!dst || !src) return GQA_ERR_INVALID_ARG;
+  const int elt = dtype == GQA_F32 ? 4 : 2;
+  const int vec = 16 / elt;
+  const int sms = sm_count(current_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  if (inner % vec == 0 && aligned16(dst) && aligned16(src)) {
+    const long long work = outer * K * (inner / vec);
+    const int grid = grid_for(work, 256, sms);
+    if (dtype == GQA_BF16)
+      gqa::meanpool_vec_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+          static_cast<uint4*>(dst), static_cast<const uint4*>(src), outer, H, K, inner / vec);
+    else
+      gqa::meanpool_vec_kernel<float><<<grid, 256, 0, st>>>(static_cast<uint4*>(dst),
+                                                            static_cast<const uint4*>(src), outer, H, K, inner / vec);
+  } else {
+    if ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & (uintptr_t)(elt - 1))
+      return GQA_ERR_ALIGN;
+    const long long work = outer * K * inner;
+    const int grid = grid_for(work, 256, sms);
+    if (dtype == GQA_BF16)
+      gqa::meanpool_scalar_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+          static_cast<__nv_bfloat16*>(dst), static_cast<const __nv_bfloat16*>(src), outer, H, K, inner);
+    else
+      gqa::meanpool_scalar_kernel<float><<<grid, 256, 0, st>>>(static_cast<float*>(dst),
+                                                               static_cast<const float*>(src), outer, H, K, inner);
+  }
+  return launch_status();
+}
+
+int gqa_get_last_error(gqa_stream_t stream, uint32_t* bits) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GQA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, gqa::g_error_word, sizeof(v)) != cudaSuccess) return GQA_ERR_CUDA;
+  if (v) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(gqa::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return GQA_ERR_CUDA;
+  }
+  if (bits) *bits = v;
+  return v ? GQA_ERR_DEVICE : GQA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,149 @@
+"""ctypes binding of libgqa.so (include/gqa.h), same names as the C ABI.
+
+Argument marshalling only: each function takes torch tensors that already
+live on the GPU, checks their shapes against one another, and passes raw
+pointers, sizes and the current CUDA stream to the library. Every step of the
+computation runs in the library's CUDA kernels; there is no other code path.
+If the library is missing the import fails with an error naming the build
+command.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgqa.so")
+
+GQA_F32, GQA_BF16 = 0, 1
+GQA_OK = 0
+GQA_ERR_DEVICE = -5
+GQA_ERR_UNSUPPORTED = -6
+GQA_DEVERR_APPEND_POS, GQA_DEVERR_SEQLEN, GQA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
+
+EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode", "gqa_prefill_causal",
+            "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string")
+
+
+class GqaError(RuntimeError):
+    def __init__(self, fn: str, status: int, bits: int = 0):
+        self.status, self.bits = status, bits
+        name = _lib.gqa_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{fn}: {name} ({status})" + (f", device error bits 0x{bits:x}" if bits else ""))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_02_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    lib.gqa_kv_append.restype = I
+    lib.gqa_kv_append.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+    lib.gqa_decode_workspace_bytes.restype = SZ
+    lib.gqa_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.gqa_decode.restype = I
+    lib.gqa_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, I, P]
+    lib.gqa_prefill_causal.restype = I
+    lib.gqa_prefill_causal.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.gqa_meanpool_kv.restype = I
+    lib.gqa_meanpool_kv.argtypes = [P, P, I64, I, I, I64, I, P]
+    lib.gqa_get_last_error.restype = I
+    lib.gqa_get_last_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.gqa_status_string.restype = ctypes.c_char_p
+    lib.gqa_status_string.argtypes = [I]
+    return lib
+
+
+_lib = _load()
+
+
+def library():
+    """The loaded ctypes handle (for tests that call the C ABI directly)."""
+    return _lib
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GQA_BF16
+    if t.dtype == torch.float32:
+        return GQA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: bfloat16 or float32")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on the GPU")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(fn: str, status: int):
+    if status != GQA_OK:
+        raise GqaError(fn, status)
+
+
+def gqa_kv_append(k_cache, v_cache, k_new, v_new, pos, stream=None) -> None:
+    """k_cache/v_cache [B,K,S_max,d] (in place), k_new/v_new [B,K,d], pos [B] int32."""
+    B, K, S_max, d = k_cache.shape
+    assert v_cache.shape == k_cache.shape and k_new.shape == (B, K, d) and v_new.shape == (B, K, d)
+    assert pos.dtype == torch.int32 and pos.shape == (B,)
+    _check("gqa_kv_append", _lib.gqa_kv_append(_ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new), _ptr(pos),
+                                               B, K, S_max, d, _dtype(k_cache), _stream(stream)))
+
+
+def gqa_decode_workspace_bytes(B: int, H: int, K: int, S_max: int, d: int, num_splits: int = 0) -> int:
+    return int(_lib.gqa_decode_workspace_bytes(B, H, K, S_max, d, num_splits))
+
+
+def gqa_decode(out, q, k_cache, v_cache, seqlens, scale: float, num_splits: int = 0, workspace=None,
+               stream=None) -> None:
+    """out/q [B,H,d], k_cache/v_cache [B,K,S_max,d], seqlens [B] int32; workspace a uint8 tensor."""
+    B, H, d = q.shape
+    _, K, S_max, _ = k_cache.shape
+    assert out.shape == q.shape and k_cache.shape[0] == B and k_cache.shape[3] == d
+    assert v_cache.shape == k_cache.shape and seqlens.dtype == torch.int32 and seqlens.shape == (B,)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("gqa_decode", _lib.gqa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, H, K,
+                                         S_max, d, float(scale), int(num_splits), _ptr(workspace), ws_bytes,
+                                         _dtype(q), _stream(stream)))
+
+
+def gqa_prefill_causal(out, q, k, v, scale: float, k_cache=None, v_cache=None, stream=None) -> None:
+    """out/q [B,S,H,d], k/v [B,S,K,d]; optional caches [B,K,S_max,d] get rows 0..S-1."""
+    B, S, H, d = q.shape
+    K = k.shape[2]
+    assert out.shape == q.shape and k.shape == (B, S, K, d) and v.shape == k.shape
+    S_max = k_cache.shape[2] if k_cache is not None else S
+    if k_cache is not None:
+        assert k_cache.shape == (B, K, S_max, d) and v_cache is not None and v_cache.shape == k_cache.shape
+    _check("gqa_prefill_causal", _lib.gqa_prefill_causal(_ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache),
+                                                         _ptr(v_cache), B, S, H, K, S_max, d, float(scale),
+                                                         _dtype(q), _stream(stream)))
+
+
+def gqa_meanpool_kv(dst, src, stream=None) -> None:
+    """src [outer, H, inner] -> dst [outer, K, inner]."""
+    outer, H, inner = src.shape
+    K = dst.shape[1]
+    assert dst.shape == (outer, K, inner)
+    _check("gqa_meanpool_kv", _lib.gqa_meanpool_kv(_ptr(dst), _ptr(src), outer, H, K, inner, _dtype(src),
+                                                   _stream(stream)))
+
+
+def gqa_get_last_error(stream=None) -> Tuple[int, int]:
+    """(status, bits): synchronises the stream, reads and clears the device error word."""
+    bits = ctypes.c_uint32(0)
+    status = _lib.gqa_get_last_error(_stream(stream), ctypes.byref(bits))
+    return int(status), int(bits.value)

@@ -1,0 +1,127 @@
+"""The C ABI on the host: the library loads, exports every symbol that
+include/gqa.h declares, and rejects bad arguments before touching the GPU.
+Also checks that the oracle and the CUDA path share no code."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kv_cache_02_b200 import build
+
+    build.build()
+    from kv_cache_02_b200 import gqa
+
+    return gqa.library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GQA_API\s+[\w\s\*]+?\b(gqa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_symbols() == sorted(["gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode",
+                                         "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_last_error",
+                                         "gqa_status_string"])
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_binding_names_match_the_c_abi():
+    from kv_cache_02_b200 import gqa
+
+    for name in declared_symbols():
+        if name == "gqa_status_string":
+            continue
+        assert callable(getattr(gqa, name)), name
+
+
+def test_status_strings(lib):
+    assert lib.gqa_status_string(0) == b"GQA_OK"
+    assert lib.gqa_status_string(-2) == b"GQA_ERR_SHAPE"
+    assert lib.gqa_status_string(-99) == b"GQA_ERR_UNKNOWN"
+
+
+P = 0x10000  # a fake, 16-byte-aligned device address: never dereferenced by these calls
+
+
+def test_decode_rejects_bad_arguments(lib):
+    f = lib.gqa_decode
+    # H % K != 0
+    assert f(P, P, P, P, P, 1, 6, 4, 16, 64, 1.0, 0, None, 0, 1, None) == -2
+    # unsupported head dim
+    assert f(P, P, P, P, P, 1, 8, 2, 16, 96, 1.0, 0, None, 0, 1, None) == -2
+    # bad dtype
+    assert f(P, P, P, P, P, 1, 8, 2, 16, 64, 1.0, 0, None, 0, 7, None) == -1
+    # negative split count
+    assert f(P, P, P, P, P, 1, 8, 2, 16, 64, 1.0, -1, None, 0, 1, None) == -1
+    # NULL pointer
+    assert f(None, P, P, P, P, 1, 8, 2, 16, 64, 1.0, 0, None, 0, 1, None) == -1
+    # misaligned pointer
+    assert f(P + 2, P, P, P, P, 1, 8, 2, 16, 64, 1.0, 0, None, 0, 1, None) == -3
+    # empty batch is a no-op
+    assert f(None, None, None, None, None, 0, 8, 2, 16, 64, 1.0, 0, None, 0, 1, None) == 0
+    # TMA row coordinates are int32: B*K*S_max must stay below 2^31
+    assert f(P, P, P, P, P, 1 << 12, 8, 8, 1 << 16, 128, 1.0, 0, None, 0, 1, None) == -2
+
+
+def test_append_and_meanpool_reject_bad_arguments(lib):
+    assert lib.gqa_kv_append(P, P, P, P, P, 2, 2, 8, 72, 1, None) == -2
+    assert lib.gqa_kv_append(P, P, P + 8, P, P, 2, 2, 8, 64, 1, None) == -3
+    assert lib.gqa_kv_append(None, P, P, P, P, 2, 2, 8, 64, 1, None) == -1
+    assert lib.gqa_kv_append(None, None, None, None, None, 0, 2, 8, 64, 1, None) == 0
+    assert lib.gqa_meanpool_kv(P, P, 1, 6, 4, 64, 1, None) == -2
+    assert lib.gqa_meanpool_kv(P, P, -1, 8, 4, 64, 1, None) == -1
+    assert lib.gqa_meanpool_kv(None, None, 0, 8, 4, 64, 1, None) == 0
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    f = lib.gqa_prefill_causal
+    assert f(P, P, P, P, None, None, 1, 16, 6, 4, 16, 128, 1.0, 1, None) == -2
+    assert f(P, P, P, P, P, None, 1, 16, 8, 4, 16, 128, 1.0, 1, None) == -1   # one cache pointer only
+    assert f(P, P, P, P, P, P, 1, 32, 8, 4, 16, 128, 1.0, 1, None) == -2      # S > S_max
+    assert f(P, P, P, P, None, None, 1, 16, 8, 4, 16, 128, 1.0, 0, None) == -6  # f32 prefill
+    assert f(None, None, None, None, None, None, 0, 16, 8, 4, 16, 128, 1.0, 1, None) == 0
+
+
+def test_workspace_size_is_zero_for_invalid_shapes(lib):
+    assert lib.gqa_decode_workspace_bytes(1, 6, 4, 16, 64, 0) == 0
+    assert lib.gqa_decode_workspace_bytes(1, 8, 2, 16, 80, 0) == 0
+    # long single sequence: the key axis is split, partials need room
+    assert lib.gqa_decode_workspace_bytes(1, 64, 8, 131072, 128, 0) > 0
+
+
+def _python_imports(path):
+    out = set()
+    for line in open(path, encoding="utf-8"):
+        m = re.match(r"\s*(?:from|import)\s+([\w\.]+)", line)
+        if m:
+            out.add(m.group(1).split(".")[0])
+    return out
+
+
+def test_oracle_and_cuda_path_share_no_code():
+    pkg = os.path.join(ROOT, "kv_cache_02_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            p = os.path.join(dirpath, f)
+            if f.endswith(".py"):
+                assert "oracle" not in _python_imports(p), p
+            if f.endswith((".cu", ".cuh", ".h", ".c")):
+                assert "oracle" not in open(p, encoding="utf-8").read().lower(), p
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        p = os.path.join(ROOT, "oracle", f)
+        if f.endswith(".py"):
+            assert "kv_cache_02_b200" not in _python_imports(p), p
+        if f.endswith(".c"):
+            assert "#include \"" not in open(p, encoding="utf-8").read(), p

@@ -1,0 +1,147 @@
+"""GPU parity of gqa_decode with the float64 oracle.
+
+Small shapes are compared element by element (several tiles, ragged tails,
+NaN in every cache row past a sequence's length). The full-size workloads run
+in the launch configuration the benchmark times and are compared on sampled
+(b, h) rows, which the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from _helpers import Guarded, assert_close, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def gqa():
+    from kv_cache_02_b200 import gqa as g
+
+    return g
+
+
+def run_decode(gqa, inp, scale, num_splits=0, guarded=True):
+    q = dev(inp["q"])
+    kc, vc = dev(inp["k_cache"]), dev(inp["v_cache"])
+    lens = dev(inp["seqlens"].astype(np.int32))
+    B, H, d = inp["q"].shape
+    K, S_max = inp["k_cache"].shape[1], inp["k_cache"].shape[2]
+    ws_bytes = gqa.gqa_decode_workspace_bytes(B, H, K, S_max, d, num_splits)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+    out = Guarded((B, H, d), q.dtype)
+    gqa.gqa_decode(out.t, q, kc, vc, lens, scale, num_splits, ws if ws_bytes else None)
+    status = gqa.gqa_get_last_error()
+    assert out.intact(), "write outside the output buffer"
+    return host(out.t), status
+
+
+def make(B, H, K, d, S_max, lens, dtype, seed):
+    lens = np.asarray(lens, np.int32)
+    return {
+        "q": synth.normal((B, H, d), dtype, seed, 1),
+        "k_cache": synth.cache(B * K, S_max, d, dtype, seed, 2, lens, K).reshape(B, K, S_max, d),
+        "v_cache": synth.cache(B * K, S_max, d, dtype, seed, 3, lens, K).reshape(B, K, S_max, d),
+        "seqlens": lens,
+    }
+
+
+SMALL = [
+    # B, H, K, d, S_max, lens
+    (3, 16, 4, 128, 300, (300, 1, 77)),          # G = 4, ragged, one-row sequence
+    (4, 64, 8, 128, 1000, (0, 999, 1000, 513)),   # G = 8, an empty sequence
+    (2, 8, 8, 64, 200, (200, 65)),                # G = 1 (MHA), d = 64
+    (2, 64, 1, 128, 700, (700, 129)),             # G = 64 (MQA): eight head slices
+    (2, 12, 2, 64, 150, (150, 16)),               # G = 6
+    (1, 24, 2, 128, 333, (333,)),                 # G = 12: slices of 8 and 4 heads
+]
+
+
+@pytest.mark.parametrize("num_splits", [0, 1, 3])
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: f"B{s[0]}H{s[1]}K{s[2]}d{s[3]}S{s[4]}")
+def test_decode_bf16_small(gqa, shape, num_splits):
+    B, H, K, d, S_max, lens = shape
+    inp = make(B, H, K, d, S_max, lens, synth.BF16, 0xDEC0 + B * 31 + H + K + d)
+    scale = 1.0 / np.sqrt(d)
+    got, status = run_decode(gqa, inp, scale, num_splits)
+    assert status == (0, 0)
+    ref = oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], scale)
+    assert_close(got, ref, f"{shape} splits={num_splits}")
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert np.all(oracle.widen(got[b]) == 0.0)
+
+
+@pytest.mark.parametrize("num_splits", [0, 1, 4])
+def test_decode_f32_tiny_workload(gqa, num_splits):
+    w = synth.DECODE_WORKLOADS["tiny_decode_b1_h8_k2_d64_s128_f32"]
+    inp = synth.decode_inputs(w)
+    scale = 1.0 / np.sqrt(w.d)
+    got, status = run_decode(gqa, inp, scale, num_splits)
+    assert status == (0, 0)
+    ref = oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], scale)
+    assert_close(got, ref, "tiny f32")
+
+
+@pytest.mark.parametrize("shape", [(3, 64, 2, 128, 200, (200, 0, 31)), (2, 8, 4, 64, 90, (90, 40))])
+def test_decode_f32_ragged(gqa, shape):
+    B, H, K, d, S_max, lens = shape
+    inp = make(B, H, K, d, S_max, lens, synth.F32, 0xF320 + H)
+    got, status = run_decode(gqa, inp, 0.1, 2)
+    assert status == (0, 0)
+    assert_close(got, oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], 0.1), str(shape))
+
+
+def test_decode_split_counts_agree(gqa):
+    inp = make(2, 32, 8, 128, 2048, (2048, 1500), synth.BF16, 0x5A5A)
+    ref = oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], 0.088)
+    outs = []
+    for ns in (1, 2, 7, 32):
+        got, status = run_decode(gqa, inp, 0.088, ns)
+        assert status == (0, 0)
+        assert_close(got, ref, f"splits={ns}")
+        outs.append(oracle.widen(got))
+    for o in outs[1:]:
+        assert np.max(np.abs(o - outs[0])) < 2e-2
+
+
+def test_decode_bad_length_reported_and_zeroed(gqa):
+    inp = make(3, 16, 4, 128, 64, (64, 64, 10), synth.BF16, 0xBAD)
+    inp["seqlens"] = np.array([64, 65, 10], np.int32)  # 65 > S_max
+    got, (status, bits) = run_decode(gqa, inp, 0.1)
+    assert status == gqa.GQA_ERR_DEVICE and bits & gqa.GQA_DEVERR_SEQLEN
+    assert np.all(oracle.widen(got[1]) == 0.0)
+    ok = np.array([64, 0, 10], np.int32)
+    ref = oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], ok, 0.1)
+    assert_close(got[[0, 2]], ref[[0, 2]], "valid rows next to a bad one")
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, launch configuration of the benchmark, sampled rows
+
+FULL = ["llama3_8b_decode_b8_h32_k8_d128_s8192", "ragged_70b_decode_b32_h64_k8_d128_s1k_16k",
+        "long_ctx_gqa_b1_h64_k8_d128_s131072", "long_ctx_mqa_b1_h64_k1_d128_s131072"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_decode_full_size_sampled(gqa, name):
+    w = synth.DECODE_WORKLOADS[name]
+    inp = synth.decode_inputs(w)
+    if w.append:
+        # the benchmark's step: append the new token at pos, then decode over pos + 1 rows
+        kc, vc = oracle.kv_append(inp["k_cache"], inp["v_cache"], inp["k_new"], inp["v_new"], inp["pos"])
+        tk, tv = dev(inp["k_cache"]), dev(inp["v_cache"])
+        gqa.gqa_kv_append(tk, tv, dev(inp["k_new"]), dev(inp["v_new"]), dev(inp["pos"]))
+        assert np.array_equal(host(tk), kc) and np.array_equal(host(tv), vc)
+        inp["k_cache"], inp["v_cache"] = kc, vc
+    scale = 1.0 / np.sqrt(w.d)
+    got, status = run_decode(gqa, inp, scale, 0)
+    assert status == (0, 0)
+    assert np.all(np.isfinite(oracle.widen(got)))
+    rng = np.random.default_rng(7)
+    sel = np.stack([rng.integers(0, w.B, 48), rng.integers(0, w.H, 48)], 1)
+    sel = np.concatenate([sel, [[0, 0], [w.B - 1, w.H - 1]]]).astype(np.int32)
+    ref = oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], scale, sel=sel)
+    assert_close(got[sel[:, 0], sel[:, 1]], ref, name)
