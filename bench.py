@@ -324,6 +324,33 @@ def extra_measurements(args):
                      "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "l2": "flushed (512 MiB write)"}
         del q, kc, vc, out, ws, flush
         torch.cuda.empty_cache()
+    # causal prefill with the KV-cache write: FLOPs over the causal pairs (j <= i) only
+    w = synth.PREFILL_WORKLOADS["causal_prefill_b4_s4096_h32_k8_d128"]
+    inp = synth.prefill_inputs(w)
+
+    def to_dev2(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).cuda()
+
+    q, k, v = to_dev2(inp["q"]), to_dev2(inp["k"]), to_dev2(inp["v"])
+    out = torch.empty_like(q)
+    kc = torch.empty((w.B, w.K, w.S, w.d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    flops = 4.0 * w.B * w.H * w.d * w.S * (w.S + 1) / 2
+    times = []
+    for it in range(args.warmup + 20):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        gqa.gqa_prefill_causal(out, q, k, v, 1.0 / np.sqrt(w.d), kc, vc)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    tf = flops / (ms * 1e-3) / 1e12
+    res[w.name] = {"ms": round(ms, 4), "flops": flops, "TFLOP/s": round(tf, 1),
+                   "frac_of_measured_bf16_burst": round(tf / peaks["bf16_tflops"], 4),
+                   "frac_of_measured_bf16_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                   "includes": "attention + KV-cache write"}
     if gqa.gqa_get_last_error() != (0, 0):
         raise RuntimeError("device error in extra measurements")
     return res

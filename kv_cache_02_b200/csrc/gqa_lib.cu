@@ -156,12 +156,31 @@ int launch_decode_f32(const DecodePlan& pl, const DecodeParams& p, const void* k
   return launch_status();
 }
 
+int launch_prefill(void* out, const void* q, const void* k, const void* v, void* k_cache, void* v_cache, int B, int S,
+                   int H, int K, int S_max, int d, float scale, cudaStream_t st, int sms);
+
 int grid_for(long long work_items, int threads, int sms) {
   long long blocks = (work_items + threads - 1) / threads;
   long long cap = (long long)sms * 16;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   return (int)blocks;
+}
+
+int launch_prefill(void* out, const void* q, const void* k, const void* v, void* k_cache, void* v_cache, int B, int S,
+                   int H, int K, int S_max, int d, float scale, cudaStream_t st, int sms) {
+  auto fn = reinterpret_cast<gqa::PfEncodeFn>(encode_fn());
+  if (!fn) return GQA_ERR_CUDA;
+  if ((long long)B * S >= (1ll << 31)) return GQA_ERR_SHAPE;
+  int rc = d == 128 ? gqa::launch_prefill_d<128>(fn, out, q, k, v, B, S, H, K, scale, st)
+                    : gqa::launch_prefill_d<64>(fn, out, q, k, v, B, S, H, K, scale, st);
+  if (rc != GQA_OK || !k_cache) return rc;
+  const int cpr = d * 2 / 16;
+  const long long work = 2ll * B * S * K * cpr;
+  gqa::kv_write_prompt_kernel<<<grid_for(work, 256, sms), 256, 0, st>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
+      static_cast<const uint4*>(v), B, S, K, S_max, cpr);
+  return launch_status();
 }
 
 }  // namespace
@@ -276,8 +295,8 @@ int gqa_prefill_causal(void* out, const void* q, const void* k, const void* v, v
   if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return GQA_ERR_ALIGN;
   if (k_cache && (!aligned16(k_cache) || !aligned16(v_cache))) return GQA_ERR_ALIGN;
   if (dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
-  return gqa::launch_prefill(out, q, k, v, k_cache, v_cache, B, S, H, K, S_max, d, scale, (cudaStream_t)stream,
-                             sm_count(current_device()));
+  return launch_prefill(out, q, k, v, k_cache, v_cache, B, S, H, K, S_max, d, scale, (cudaStream_t)stream,
+                        sm_count(current_device()));
 }
 
 int gqa_meanpool_kv(void* dst, const void* src, int64_t outer, int H, int K, int64_t inner, gqa_dtype dtype,

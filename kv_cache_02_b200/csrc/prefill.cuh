@@ -1,14 +1,449 @@
-// Causal GQA prefill (tcgen05 / TMEM / TMA). Not built yet: reports
-// GQA_ERR_UNSUPPORTED.
+// Causal GQA prefill on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+//   out[b, i, h, :] = sum_{j <= i} softmax_j(scale * q[b,i,h] . k[b,j,g]) v[b,j,g],  g = h / (H/K)
+//
+// One CTA computes one 128-row query tile of one head (two CTAs share an SM:
+// 112 KB of shared memory and 256 TMEM columns each). Warp roles:
+//   warps 0-3  softmax: thread r owns query row r (= TMEM lane r)
+//   warp 4     TMA producer: Q once, then 64-key K/V tiles into a 2-stage ring
+//   warp 5     MMA issuer (one thread) and TMEM allocator
+// Per key tile j:
+//   S_j = Q K_j^T   tcgen05.mma, M=128 N=64 K=d, fp32 in TMEM (two S buffers)
+//   softmax thread r: tcgen05.ld its S row, causal mask, running max m and sum
+//       l in log2 units, P = 2^(S - m) as bf16 into shared memory (128-byte
+//       swizzled, the K-major operand layout)
+//   O += P V_j      tcgen05.mma, M=128 N=d K=64, fp32 accumulator in TMEM
+// The accumulator is rescaled only when a row's maximum grows by more than
+// 2^8 (until then P <= 256, exact enough in fp32 and bf16), so most tiles
+// touch O only through the MMA. The final O / l is written as bf16.
+//
+// Heads of one group run in adjacent CTAs, so a K/V tile read from HBM is
+// reused from L2 by the group's query heads; the heavy (late) query tiles are
+// scheduled first.
 #pragma once
 
 #include "common.cuh"
 
 namespace gqa {
 
-inline int launch_prefill(void*, const void*, const void*, const void*, void*, void*, int, int, int, int, int, int,
-                          float, cudaStream_t, int) {
-  return GQA_ERR_UNSUPPORTED;
+constexpr int kPfBM = 128;  // query rows per CTA
+constexpr int kPfBN = 64;   // keys per tile
+constexpr int kPfStages = 2;
+constexpr int kPfThreads = 192;
+constexpr int kPfTmemCols = 256;
+
+template <int D>
+struct PfCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kQHalf = kPfBM * 128;         // bytes of one 64-column half of Q
+  static constexpr int kKVHalf = kPfBN * 128;        // bytes of one 64-column half of a K or V tile
+  static constexpr int kQBytes = kHalves * kQHalf;
+  static constexpr int kTileBytes = kHalves * kKVHalf;
+  static constexpr int kStageBytes = 2 * kTileBytes;  // K and V
+  static constexpr int kPBytes = kPfBM * kPfBN * 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = kQBytes;
+  static constexpr int kPOff = kKVOff + kPfStages * kStageBytes;
+  static constexpr int kBarOff = kPOff + kPBytes;
+  static constexpr int kNumBars = 1 + 2 * kPfStages + 2 + 2 + 1 + 1 + 1;
+  // at most two CTAs per SM (their 2 x 256 TMEM columns fill the SM's 512)
+  static constexpr int kSmemBytes = (kBarOff + kNumBars * 8 + 16) > 80 * 1024 ? (kBarOff + kNumBars * 8 + 16)
+                                                                               : 80 * 1024;
+  static constexpr int kOCol = 2 * kPfBN;  // TMEM column of O (after the two S buffers)
+  static_assert(kOCol + D <= kPfTmemCols, "TMEM budget");
+};
+
+// ---------------------------------------------------------------------------
+// tcgen05 wrappers
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* holder, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(holder)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+      "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+      "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (sm100): 128-byte swizzle, version 1.
+//   lbo/sbo in bytes: K-major -> sbo = stride between 8-row groups, lbo unused (16);
+//   MN-major -> lbo = stride between 64-element column blocks, sbo = stride between 8-row groups.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version (sm100)
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, M x N, operand majors.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                               // D format: f32
+         | (1u << 7)                             // A: bf16
+         | (1u << 10)                            // B: bf16
+         | ((a_mn_major ? 1u : 0u) << 15)        // A major
+         | ((b_mn_major ? 1u : 0u) << 16)        // B major
+         | ((uint32_t)(N >> 3) << 17)            // N / 8
+         | ((uint32_t)(M >> 4) << 24);           // M / 16
+}
+
+struct PrefillParams {
+  void* out;  // [B, S, H, D] bf16
+  int B, S, H, K, G, n_qt;
+  float scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kPfThreads, 2)
+    prefill_causal_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+  using C = PfCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* q_full = bars;                  // TMA Q landed
+  uint64_t* kv_full = bars + 1;             // [2] TMA K/V tile landed
+  uint64_t* kv_empty = kv_full + kPfStages; // [2] PV of that tile finished
+  uint64_t* s_full = kv_empty + kPfStages;  // [2] S buffer written by the MMA
+  uint64_t* s_free = s_full + 2;            // [2] S buffer read by all softmax threads
+  uint64_t* p_full = s_free + 2;            // P in smem (and O rescaled) for the next PV
+  uint64_t* pv_done = p_full + 1;           // the last issued PV finished
+  uint64_t* mma_done = pv_done + 1;         // every MMA of this CTA finished
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // the 128-byte swizzle pattern assumes 1024-byte aligned operand tiles
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) raise_error(GQA_DEVERR_TIMEOUT);
+    return;
+  }
+
+  // work item: heavy query tiles first; the G heads of a group are adjacent
+  const int per_qt = p.B * p.H;
+  const int qt = p.n_qt - 1 - (int)(blockIdx.x / per_qt);
+  const int rem = (int)(blockIdx.x % per_qt);
+  const int b = rem / p.H, h = rem % p.H;
+  const int g = h / p.G;
+  const int q0 = qt * kPfBM;
+  const int n_tiles = min((p.S + kPfBN - 1) / kPfBN, (q0 + kPfBM + kPfBN - 1) / kPfBN);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kPfStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_holder, kPfTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 4) {
+    // -------------------------------------------------------------- TMA
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
+      mbar_arrive_expect_tx(q_full, C::kQBytes);
+#pragma unroll
+      for (int hf = 0; hf < C::kHalves; ++hf)
+        tma_load_3d(smem + C::kQOff + hf * C::kQHalf, &tm_q, hf * 64, h, b * p.S + q0, q_full, pol_q);
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % kPfStages;
+        if (j >= kPfStages && !mbar_wait_bounded(&kv_empty[s], ((j / kPfStages) - 1) & 1)) break;
+        uint8_t* kd = smem + C::kKVOff + s * C::kStageBytes;
+        uint8_t* vd = kd + C::kTileBytes;
+        mbar_arrive_expect_tx(&kv_full[s], C::kStageBytes);
+#pragma unroll
+        for (int hf = 0; hf < C::kHalves; ++hf) {
+          tma_load_3d(kd + hf * C::kKVHalf, &tm_k, hf * 64, g, b * p.S + j * kPfBN, &kv_full[s], pol_kv);
+          tma_load_3d(vd + hf * C::kKVHalf, &tm_v, hf * 64, g, b * p.S + j * kPfBN, &kv_full[s], pol_kv);
+        }
+        ++issued;
+      }
+      for (int j = max(0, issued - kPfStages); j < issued; ++j)
+        mbar_wait_bounded(&kv_full[j % kPfStages], (j / kPfStages) & 1);
+    }
+  } else if (warp == 5) {
+    // -------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kPfBM, kPfBN, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kPfBM, D, false, true);
+      const uint32_t q_addr = smem_u32(smem + C::kQOff);
+      const uint32_t p_addr = smem_u32(smem + C::kPOff);
+      bool ok = mbar_wait_bounded(q_full, 0);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % kPfStages;
+        if (!mbar_wait_bounded(&kv_full[s], (j / kPfStages) & 1)) return false;
+        if (j >= 2 && !mbar_wait_bounded(&s_free[j & 1], ((j >> 1) - 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + C::kKVOff + s * C::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;  // 16 columns = 32 bytes inside the 128-byte swizzle row
+          const uint64_t ad = smem_desc_sw128(q_addr + (kk >> 2) * C::kQHalf + off, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(k_addr + (kk >> 2) * C::kKVHalf + off, 16, 1024);
+          tc_mma(tmem + (uint32_t)((j & 1) * kPfBN), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[j & 1]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + 1 < n_tiles && !issue_s(j + 1)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait_bounded(p_full, j & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(smem + C::kKVOff + (j % kPfStages) * C::kStageBytes + C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kPfBN / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(p_addr + kk * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(v_addr + kk * 16 * 128, C::kKVHalf, 1024);
+          tc_mma(tmem + C::kOCol, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(pv_done);
+        tc_commit(&kv_empty[j % kPfStages]);
+      }
+      tc_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0);
+    }
+  } else {
+    // ---------------------------------------------------------- softmax
+    const int r = threadIdx.x;  // query row within the tile = TMEM lane
+    const int qpos = q0 + r;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    uint8_t* prow = smem + C::kPOff + r * 128;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      // tcgen05.ld/st are warp-collective: every decision that guards them is warp-uniform
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[j & 1], (j >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float x[64];
+      {
+        float a[32], c[32];
+        tmem_ld32(lane_addr + (uint32_t)((j & 1) * kPfBN), a);
+        tmem_ld32(lane_addr + (uint32_t)((j & 1) * kPfBN + 32), c);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x[i] = a[i];
+          x[32 + i] = c[i];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[j & 1]);
+
+      const int k0 = j * kPfBN;
+      const int kmax = min(qpos, p.S - 1) - k0;  // keys k0 + c with c <= kmax are visible
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        x[c] = c <= kmax ? x[c] * p.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, x[c]);
+      }
+      float alpha = 1.f;
+      bool rescale = false;
+      if (mt > m_used + 8.f) {  // first tile: m_used = -inf
+        const float m_new = fmaxf(mt, m_used);
+        alpha = fast_exp2(m_used - m_new);
+        rescale = j > 0;
+        m_used = m_new;
+      }
+      float sum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = fast_exp2(x[2 * c] - m_used);
+        const float p1 = fast_exp2(x[2 * c + 1] - m_used);
+        sum += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l = l * alpha + sum;
+      // P buffer and O are free once the previous tile's PV has finished
+      if (j > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, (j - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, rescale)) {  // lanes that keep their max scale by alpha = 1
+#pragma unroll 1
+        for (int cb = 0; cb < D; cb += 32) {
+          float o[32];
+          tmem_ld32(lane_addr + C::kOCol + cb, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(lane_addr + C::kOCol + cb, o);
+        }
+        tc_wait_st();
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t off = ((uint32_t)(c ^ (r & 7))) << 4;
+        *reinterpret_cast<uint4*>(prow + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_async_shared();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // epilogue: O / l -> bf16
+    if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(pv_done, (n_tiles - 1) & 1))) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+      uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)b * p.S + qpos) * p.H + h) * D);
+#pragma unroll 1
+      for (int cb = 0; cb < D; cb += 32) {
+        float o[32];
+        tmem_ld32(lane_addr + C::kOCol + cb, o);
+        tc_wait_ld();
+        if (qpos < p.S) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[cb / 8 + i] = make_uint4(pack_bf16x2(o[8 * i] * inv_l, o[8 * i + 1] * inv_l),
+                                         pack_bf16x2(o[8 * i + 2] * inv_l, o[8 * i + 3] * inv_l),
+                                         pack_bf16x2(o[8 * i + 4] * inv_l, o[8 * i + 5] * inv_l),
+                                         pack_bf16x2(o[8 * i + 6] * inv_l, o[8 * i + 7] * inv_l));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kPfTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host launch
+
+typedef CUresult (*PfEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// [B*S, heads, D] bf16 viewed as (x = D, y = heads, z = B*S); box 64 x 1 x rows
+inline bool encode_bsh(PfEncodeFn fn, CUtensorMap* map, const void* base, uint64_t BS, uint64_t heads, uint64_t Dd,
+                       uint32_t rows) {
+  cuuint64_t dims[3] = {Dd, heads, BS};
+  cuuint64_t strides[2] = {Dd * 2, heads * Dd * 2};
+  cuuint32_t box[3] = {64, 1, rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch_prefill_d(PfEncodeFn fn, void* out, const void* q, const void* k, const void* v, int B, int S, int H,
+                     int K, float scale, cudaStream_t st) {
+  using C = PfCfg<D>;
+  CUtensorMap tq, tk, tv;
+  if (!encode_bsh(fn, &tq, q, (uint64_t)B * S, H, D, kPfBM) || !encode_bsh(fn, &tk, k, (uint64_t)B * S, K, D, kPfBN) ||
+      !encode_bsh(fn, &tv, v, (uint64_t)B * S, K, D, kPfBN))
+    return GQA_ERR_CUDA;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    if (cudaFuncSetAttribute(prefill_causal_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      return GQA_ERR_CUDA;
+    configured[dev] = true;
+  }
+  PrefillParams p;
+  p.out = out;
+  p.B = B;
+  p.S = S;
+  p.H = H;
+  p.K = K;
+  p.G = H / K;
+  p.n_qt = (S + kPfBM - 1) / kPfBM;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long grid = (long long)p.n_qt * B * H;
+  prefill_causal_kernel<D><<<(unsigned)grid, kPfThreads, C::kSmemBytes, st>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 }  // namespace gqa
