@@ -57,7 +57,8 @@ typedef enum {
   GQA_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
   GQA_ERR_CUDA = -4,        /* a CUDA call or kernel launch failed */
   GQA_ERR_DEVICE = -5,      /* the device error word was set (see GQA_DEVERR_*) */
-  GQA_ERR_UNSUPPORTED = -6  /* valid request that this build does not implement (e.g. f32 prefill) */
+  GQA_ERR_UNSUPPORTED = -6, /* valid request that this build does not implement (e.g. f32 prefill) */
+  GQA_ERR_SCRATCH_LIMIT = -7 /* gqa_decode_noalloc: needs more than GQA_NOALLOC_SCRATCH_BYTES of scratch */
 } gqa_status;
 
 /* Bits of the device error word. */
@@ -122,6 +123,40 @@ GQA_API size_t gqa_decode_workspace_bytes(int B, int H, int K, int S_max, int d,
 GQA_API int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
                int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
                gqa_dtype dtype, gqa_stream_t stream);
+
+/*
+ * gqa_decode_noalloc - gqa_decode without a caller-supplied workspace.
+ *
+ * The paper has no counterpart to this call. It is for callers that cannot
+ * allocate device memory when they decode, such as a plugin inside a host
+ * framework that owns all device memory through its own allocator (a raw
+ * cudaMalloc would bypass that allocator's budget), or a latency-critical
+ * serving loop that allows no allocation after start-up (cudaMalloc and
+ * cudaFree can synchronise the whole device). Such a caller still passes
+ * out, q, the caches and seqlens exactly as for gqa_decode.
+ *
+ * The split-KV partial results go to a scratch array the library holds
+ * itself: GQA_NOALLOC_SCRATCH_BYTES of static device memory on every GPU that
+ * loads the library, kept until the process exits. The call itself allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *  - A request whose partials need more than GQA_NOALLOC_SCRATCH_BYTES (what
+ *    gqa_decode_workspace_bytes reports for the same shape and num_splits)
+ *    is rejected with GQA_ERR_SCRATCH_LIMIT before anything is launched; a
+ *    smaller num_splits needs less scratch.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current). Make that first call
+ *    before any stream capture begins on the device.
+ *  - Every call on a device uses the same array, which keeps whatever the
+ *    last call left in it. Calls that overlap on the GPU (unordered streams)
+ *    race on it and produce wrong results: order them on one stream or with
+ *    events. Nothing in it has to start at zero; within one call every
+ *    partial is written before it is read.
+ *  - Arguments, results and errors are otherwise those of gqa_decode.
+ */
+#define GQA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+GQA_API int gqa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* seqlens, int B, int H, int K, int S_max, int d, float scale,
+                               int num_splits, gqa_dtype dtype, gqa_stream_t stream);
 
 /*
  * gqa_prefill_causal - causal self-attention over a whole prompt, and the

@@ -13,6 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libgqa.so")
 MAIN = os.path.join(HERE, "csrc", "gqa_lib.cu")
+UNITS = [MAIN, os.path.join(HERE, "csrc", "decode_noalloc.cu")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -36,7 +37,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not (force or stale):
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-o", tmp, MAIN]
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-o", tmp, *UNITS]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)

@@ -199,6 +199,7 @@ const char* gqa_status_string(int status) {
     case GQA_ERR_CUDA: return "GQA_ERR_CUDA";
     case GQA_ERR_DEVICE: return "GQA_ERR_DEVICE";
     case GQA_ERR_UNSUPPORTED: return "GQA_ERR_UNSUPPORTED";
+    case GQA_ERR_SCRATCH_LIMIT: return "GQA_ERR_SCRATCH_LIMIT";
     default: return "GQA_ERR_UNKNOWN";
   }
 }

@@ -24,7 +24,10 @@ GQA_ERR_DEVICE = -5
 GQA_ERR_UNSUPPORTED = -6
 GQA_DEVERR_APPEND_POS, GQA_DEVERR_SEQLEN, GQA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
-EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode", "gqa_prefill_causal",
+GQA_ERR_SCRATCH_LIMIT = -7
+GQA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
+
+EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode", "gqa_decode_noalloc", "gqa_prefill_causal",
             "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string")
 
 
@@ -46,6 +49,8 @@ def _load():
     lib.gqa_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.gqa_decode.restype = I
     lib.gqa_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, I, P]
+    lib.gqa_decode_noalloc.restype = I
+    lib.gqa_decode_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, P]
     lib.gqa_prefill_causal.restype = I
     lib.gqa_prefill_causal.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gqa_meanpool_kv.restype = I
@@ -118,6 +123,23 @@ def gqa_decode(out, q, k_cache, v_cache, seqlens, scale: float, num_splits: int 
     _check("gqa_decode", _lib.gqa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, H, K,
                                          S_max, d, float(scale), int(num_splits), _ptr(workspace), ws_bytes,
                                          _dtype(q), _stream(stream)))
+
+
+def gqa_decode_noalloc(out, q, k_cache, v_cache, seqlens, scale: float, num_splits: int = 0, stream=None) -> None:
+    """gqa_decode with the library's own static scratch instead of a caller workspace.
+
+    For callers that cannot allocate device memory at decode time. Raises
+    GqaError(GQA_ERR_SCRATCH_LIMIT) when the split-KV partials of this shape
+    and split count need more than GQA_NOALLOC_SCRATCH_BYTES. Calls that
+    overlap on the GPU share the scratch and race.
+    """
+    B, H, d = q.shape
+    _, K, S_max, _ = k_cache.shape
+    assert out.shape == q.shape and k_cache.shape[0] == B and k_cache.shape[3] == d
+    assert v_cache.shape == k_cache.shape and seqlens.dtype == torch.int32 and seqlens.shape == (B,)
+    _check("gqa_decode_noalloc", _lib.gqa_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                                         _ptr(seqlens), B, H, K, S_max, d, float(scale),
+                                                         int(num_splits), _dtype(q), _stream(stream)))
 
 
 def gqa_prefill_causal(out, q, k, v, scale: float, k_cache=None, v_cache=None, stream=None) -> None:
