@@ -1,26 +1,33 @@
-// GQA decode over a KV cache (split-KV with a log-sum-exp combine).
+// GQA decode over a KV cache.
 //
-// One CTA owns one work item (b, g, split, head slice): the keys
-// [split*chunk, min(len_b, (split+1)*chunk)) of KV head g of sequence b, and up
-// to 8 query heads of that group. Every K/V row is brought from HBM once by
-// TMA and serves all the CTA's query heads ("GQA 完全拆解", section 工程实现:
-// the group's query heads share one thread block and one load of each KV
-// block).
+// Every K/V row is brought from HBM once by TMA and serves all of its group's
+// query heads ("GQA 完全拆解", section 工程实现: the group's query heads share
+// one thread block and one load of each KV block).
 //
-// bf16 path, per CTA: warp 4 is the TMA producer (64-key tiles of K and V,
-// 128-byte swizzled, a ring of mbarrier-guarded stages); warps 0..3 each own
-// 16 keys of every tile and run on the tensor cores:
+// bf16 path. A CTA has 5 warps: warp 4 is the TMA producer (64-key tiles of K
+// and V, 128-byte swizzled, in a ring of mbarrier-guarded stages); warps 0..3
+// each own 16 keys of every tile and run on the tensor cores:
 //     S^T[16 keys x 8 heads]  = K[16 x d] * Q^T[d x 8]        (mma.sync m16n8k16)
 //     online softmax over keys, per head, in fp32 (log2 domain)
 //     O^T[d x 8 heads]       += V^T[d x 16 keys] * P^T[16 x 8]
-// Keys sit in the MMA M dimension and the group's heads in N, so G = 8 fills
-// the instruction and G = 4 uses half of it. P^T is produced from the S^T
-// accumulator with movmatrix (register transpose), with no shared-memory trip.
-// The four warps' partial (m, l, O) are merged in shared memory; the CTA then
-// writes either the final output (one split) or its partial to the workspace
-// for decode_combine_kernel.
+// Keys sit in the MMA M dimension and up to 8 of the group's heads in N, so
+// G = 8 fills the instruction and G = 4 uses half of it. P^T comes from the
+// S^T accumulator through movmatrix (a register transpose). At the end of a
+// (b, g) unit the four warps' (m, l, O) are merged in shared memory.
 //
-// f32 path (small problems, float32 storage): plain FMA, one warp per head.
+// The key axis of each (b, g) unit is cut into splits of `chunk` keys; a
+// work item is (b, g, split, head slice). bf16: persistent CTAs, two per SM;
+// each CTA's producer thread takes items from a tagged atomic counter in
+// unit order and streams their tiles through its ring without a break, so a
+// work item's epilogue (merging the four warps, writing the output or the
+// split's partial) overlaps the next item's loads, and late items go to
+// whichever CTA is free. The counter word carries a per-call tag next to the
+// count, so stale or uninitialised workspace contents read as "no items
+// taken yet": the workspace needs no initialisation. Units with more than
+// one split are merged by decode_combine_kernel (log-sum-exp), launched as a
+// programmatic dependent so that its launch overlaps the decode kernel.
+//
+// f32 path (float32 storage, small problems): plain FMA, one warp per head.
 #pragma once
 
 #include "common.cuh"
@@ -40,32 +47,269 @@ struct DecCfg {
   static constexpr int kTileBytes = kDecTileKeys * D * 2;      // K (or V) tile
   static constexpr int kStages = (D == 128) ? 3 : 6;
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kBarOffset = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 1024;  // + alignment slack
-  static_assert(kDecConsumerWarps * (kDecHeadsPerCta * D + 2 * kDecHeadsPerCta) * 4 <= kBarOffset,
-                "merge scratch must fit in the stage buffers");
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  // merge scratch: per consumer warp, m and l of 8 heads, then O of 8 heads
+  static constexpr int kMergeFloats = kDecConsumerWarps * (2 * kDecHeadsPerCta + kDecHeadsPerCta * D);
+  // persistent kernel: ring, then merge/combine scratch (the ring keeps
+  // streaming while a work item's epilogue runs), stage records, barriers
+  static constexpr int kMergeOff = kRingBytes;
+  static constexpr int kInfoOff = kMergeOff + kMergeFloats * 4;
+  static constexpr int kBarOff = kInfoOff + kStages * 16;
+  static constexpr int kSmemBytes = kBarOff + 2 * kStages * 8;
 };
 
 struct DecodeParams {
   const void* q;
   void* out;
-  float* ws_o;    // [B*K*nsplit*G, D] partial O (unnormalised, relative to m)
-  float2* ws_ml;  // [B*K*nsplit*G] partial (m, l), m in log2 units
+  float* ws_o;                 // [B*K*nsplit*G, D] partial O (unnormalised, relative to m)
+  float2* ws_ml;               // [B*K*nsplit*G] partial (m, l), m in log2 units
+  unsigned long long* ws_queue;  // work-item counter of the persistent kernel: tag | count
+  int nitems;                  // B * K * nsplit * hslices
   const int32_t* seqlens;
   int B, H, K, S_max, G, hslices, chunk, nsplit;
-  float scale_log2;  // scale * log2(e)
+  unsigned long long tag;      // 40-bit, nonzero, different on every call
+  float scale_log2;            // scale * log2(e)
 };
+
+constexpr int kCntBits = 24;
+constexpr int kMaxCombineSplits = 1024;  // splits per unit the combine kernel accepts  // count field of a tagged counter (work items stay below 2^24)
+
+__device__ __forceinline__ unsigned long long atom_add_relaxed(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.add.relaxed.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ unsigned long long atom_cas_relaxed(unsigned long long* p, unsigned long long cmp,
+                                                               unsigned long long val) {
+  unsigned long long old;
+  asm volatile("atom.cas.relaxed.gpu.global.b64 %0, [%1], %2, %3;" : "=l"(old) : "l"(p), "l"(cmp), "l"(val)
+               : "memory");
+  return old;
+}
+
+// Take a ticket from a tagged counter: returns 1, 2, 3, ... in the order the
+// CTAs of the current call arrive. A word whose tag differs from the call's
+// tag counts as zero: the first arrival claims it with one compare-and-swap,
+// every later one adds to the count (the tag, in the high bits, is left
+// alone). Nothing ever waits for another CTA.
+__device__ __forceinline__ int take_ticket(unsigned long long* cnt, unsigned long long tag) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cnt);
+  for (int attempt = 0; attempt < 64; ++attempt) {
+    if ((cur >> kCntBits) == tag) return (int)((atom_add_relaxed(cnt, 1ull) & ((1ull << kCntBits) - 1)) + 1);
+    const unsigned long long prev = atom_cas_relaxed(cnt, cur, (tag << kCntBits) | 1ull);
+    if (prev == cur) return 1;
+    cur = prev;  // another CTA claimed it first (or the word changed): look again
+  }
+  raise_error(GQA_DEVERR_TIMEOUT);
+  return 0;
+}
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Work item -> (unit, split, head slice); head slice varies fastest so the
-// CTAs that read the same KV chunk for different head slices run together.
+template <typename T>
+__device__ __forceinline__ void store_out(T* dst, float v);
+template <>
+__device__ __forceinline__ void store_out<float>(float* dst, float v) {
+  *dst = v;
+}
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* dst, float v) {
+  *dst = __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ int valid_len(int len, int S_max) { return (len < 0 || len > S_max) ? 0 : len; }
+
+__device__ __forceinline__ void consumer_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumerWarps * 32) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// pieces shared by the bf16 kernels
+
+// TMA loads of one tile (rows of K and V of one unit) into ring stage `s`.
+template <int D>
+__device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* full, const CUtensorMap* tm_k,
+                                           const CUtensorMap* tm_v, int row0, int rows, uint64_t policy) {
+  using C = DecCfg<D>;
+  const int nbox = (rows + kDecBoxRows - 1) / kDecBoxRows;
+  mbar_arrive_expect_tx(full, (uint32_t)(nbox * kDecBoxRows * 128 * C::kHalves * 2));
+  for (int bx = 0; bx < nbox; ++bx) {
+#pragma unroll
+    for (int hf = 0; hf < C::kHalves; ++hf) {
+      const int off = hf * C::kHalfBytes + bx * kDecBoxRows * 128;
+      tma_load_2d(stage + off, tm_k, hf * 64, row0 + bx * kDecBoxRows, full, policy);
+      tma_load_2d(stage + C::kTileBytes + off, tm_v, hf * 64, row0 + bx * kDecBoxRows, full, policy);
+    }
+  }
+}
+
+// Q^T as the B operand (k = dims, n = heads): lane holds head lane/4, dims
+// 2*(lane%4) + {0,1} (b0) and + 8 (b1) of every 16-dim step.
+template <int D>
+__device__ __forceinline__ void load_q_frag(uint32_t (&qf)[D / 16][2], const __nv_bfloat16* q, int lane, int nh) {
+  const int hn = lane >> 2;
+  const bool hv = hn < nh;
+  const uint32_t* qrow = reinterpret_cast<const uint32_t*>(q + (size_t)(hv ? hn : 0) * D);
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const uint32_t lo = __ldg(qrow + ks * 8 + (lane & 3));
+    const uint32_t hi = __ldg(qrow + ks * 8 + 4 + (lane & 3));
+    qf[ks][0] = hv ? lo : 0u;
+    qf[ks][1] = hv ? hi : 0u;
+  }
+}
+
+// Running softmax state of one consumer warp for heads a = 2*(lane%4) and
+// b = a + 1 over the keys it has seen (log2 units).
+template <int D>
+struct WarpState {
+  float m_a, m_b, l_a, l_b;
+  float o[D / 16][4];
+  __device__ __forceinline__ void reset() {
+    m_a = m_b = -INFINITY;
+    l_a = l_b = 0.f;
+#pragma unroll
+    for (int md = 0; md < D / 16; ++md) o[md][0] = o[md][1] = o[md][2] = o[md][3] = 0.f;
+  }
+};
+
+// One warp's 16 keys (kb .. kb+15) of the tile in `stage`; `rows` keys of the
+// tile are valid (the rest may hold anything, NaN included).
+template <int D>
+__device__ __forceinline__ void warp_tile(WarpState<D>& st, const uint32_t (&qf)[D / 16][2], uint32_t stage_addr,
+                                          int kb, int rows, int lane, float scale_log2) {
+  using C = DecCfg<D>;
+  const uint32_t k_base = stage_addr;
+  const uint32_t v_base = stage_addr + C::kTileBytes;
+  // ldmatrix row/column assignment (lane -> 8x8 matrix lane/8)
+  const int k_row = kb + (lane & 7) + ((lane >> 3) & 1) * 8;  // K: (r0-7,c0-7) (r8-15,c0-7) (r0-7,c8-15) ...
+  const int k_col8 = lane >> 4;
+  const int v_row = kb + (lane & 7) + (lane >> 4) * 8;  // V^T: (d0-7,k0-7) (d8-15,k0-7) (d0-7,k8-15) ...
+  const int v_col8 = (lane >> 3) & 1;
+
+  // S^T = K * Q^T
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const int chunk = ks * 2 + k_col8;  // 16-byte chunk index along the row
+    const uint32_t addr = k_base + (chunk >> 3) * C::kHalfBytes + sw128(k_row, chunk & 7);
+    uint32_t a0, a1, a2, a3;
+    ldmatrix_x4(addr, a0, a1, a2, a3);
+    mma_bf16_16816(c, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+  }
+
+  // online softmax over this block's keys (key kb + lane/4 in c0/c1, +8 in c2/c3)
+  const int key0 = kb + (lane >> 2);
+  const bool v0 = key0 < rows, v1 = key0 + 8 < rows;
+  const float x0 = v0 ? c[0] * scale_log2 : -INFINITY;
+  const float x1 = v0 ? c[1] * scale_log2 : -INFINITY;
+  const float x2 = v1 ? c[2] * scale_log2 : -INFINITY;
+  const float x3 = v1 ? c[3] * scale_log2 : -INFINITY;
+  float mx_a = fmaxf(x0, x2), mx_b = fmaxf(x1, x3);
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+  }
+  const float mn_a = fmaxf(st.m_a, mx_a), mn_b = fmaxf(st.m_b, mx_b);
+  const float al_a = fast_exp2(st.m_a - mn_a), al_b = fast_exp2(st.m_b - mn_b);
+  st.m_a = mn_a;
+  st.m_b = mn_b;
+  const float p0 = fast_exp2(x0 - mn_a), p1 = fast_exp2(x1 - mn_b);
+  const float p2 = fast_exp2(x2 - mn_a), p3 = fast_exp2(x3 - mn_b);
+  st.l_a = st.l_a * al_a + p0 + p2;
+  st.l_b = st.l_b * al_b + p1 + p3;
+#pragma unroll
+  for (int md = 0; md < D / 16; ++md) {
+    st.o[md][0] *= al_a;
+    st.o[md][1] *= al_b;
+    st.o[md][2] *= al_a;
+    st.o[md][3] *= al_b;
+  }
+
+  // P^T (k = keys, n = heads) from the S^T accumulator layout
+  const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
+  const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
+
+  // keys of this block past the valid rows: zero their V^T entries
+  uint32_t mask_lo = 0xffffffffu, mask_hi = 0xffffffffu;
+  if (kb + 16 > rows) {
+    const int lim = rows - kb;
+    const int kk = 2 * (lane & 3);
+    mask_lo = (kk < lim ? 0x0000ffffu : 0u) | (kk + 1 < lim ? 0xffff0000u : 0u);
+    mask_hi = (kk + 8 < lim ? 0x0000ffffu : 0u) | (kk + 9 < lim ? 0xffff0000u : 0u);
+  }
+
+  // O^T += V^T * P^T
+#pragma unroll
+  for (int md = 0; md < D / 16; ++md) {
+    const int chunk = md * 2 + v_col8;
+    const uint32_t addr = v_base + (chunk >> 3) * C::kHalfBytes + sw128(v_row, chunk & 7);
+    uint32_t a0, a1, a2, a3;
+    ldmatrix_x4_trans(addr, a0, a1, a2, a3);
+    mma_bf16_16816(st.o[md], a0 & mask_lo, a1 & mask_lo, a2 & mask_hi, a3 & mask_hi, pb0, pb1);
+  }
+}
+
+// Write one warp's state into the merge scratch (after a consumer barrier).
+template <int D>
+__device__ __forceinline__ void stash_warp_state(float* merge, const WarpState<D>& st, int warp, int lane) {
+  float* red_m = merge;
+  float* red_l = red_m + kDecConsumerWarps * kDecHeadsPerCta;
+  float* ow = red_l + kDecConsumerWarps * kDecHeadsPerCta + warp * kDecHeadsPerCta * D;
+  float l_a = st.l_a, l_b = st.l_b;
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, off);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, off);
+  }
+  const int ha = 2 * (lane & 3);
+  if (lane < 4) {
+    red_m[warp * 8 + ha] = st.m_a;
+    red_m[warp * 8 + ha + 1] = st.m_b;
+    red_l[warp * 8 + ha] = l_a;
+    red_l[warp * 8 + ha + 1] = l_b;
+  }
+  const int dr = lane >> 2;
+#pragma unroll
+  for (int md = 0; md < D / 16; ++md) {
+    ow[ha * D + md * 16 + dr] = st.o[md][0];
+    ow[(ha + 1) * D + md * 16 + dr] = st.o[md][1];
+    ow[ha * D + md * 16 + dr + 8] = st.o[md][2];
+    ow[(ha + 1) * D + md * 16 + dr + 8] = st.o[md][3];
+  }
+}
+
+// Merge the four warps' states for output (h, dim): returns (M, L, O).
+template <int D>
+__device__ __forceinline__ void merged(const float* merge, int h, int dim, float& M, float& L, float& O) {
+  const float* red_m = merge;
+  const float* red_l = red_m + kDecConsumerWarps * kDecHeadsPerCta;
+  const float* red_o = red_l + kDecConsumerWarps * kDecHeadsPerCta;
+  M = -INFINITY;
+#pragma unroll
+  for (int ww = 0; ww < kDecConsumerWarps; ++ww) M = fmaxf(M, red_m[ww * 8 + h]);
+  L = 0.f;
+  O = 0.f;
+#pragma unroll
+  for (int ww = 0; ww < kDecConsumerWarps; ++ww) {
+    const float f = fast_exp2(red_m[ww * 8 + h] - M);
+    L += red_l[ww * 8 + h] * f;
+    O += red_o[(ww * kDecHeadsPerCta + h) * D + dim] * f;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// fixed splits: one CTA per (b, g, split, head slice)
+
 struct DecItem {
   int b, g, unit, split, hsl, len, t_begin, t_end, h0, nh;
 };
 
+// Work item -> (unit, split, head slice); head slice varies fastest so the
+// CTAs that read the same KV chunk for different head slices run together.
 __device__ __forceinline__ DecItem decode_item(const DecodeParams& p, int heads_per_cta) {
   DecItem it;
   const int item = blockIdx.x;
@@ -88,46 +332,80 @@ __device__ __forceinline__ DecItem decode_item(const DecodeParams& p, int heads_
   return it;
 }
 
-template <typename T>
-__device__ __forceinline__ void store_out(T* dst, float v);
-template <>
-__device__ __forceinline__ void store_out<float>(float* dst, float v) {
-  *dst = v;
-}
-template <>
-__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* dst, float v) {
-  *dst = __float2bfloat16_rn(v);
+// ---------------------------------------------------------------------------
+// bf16: persistent CTAs (two per SM). The producer thread takes work items
+// (unit, split, head slice) from a tagged atomic counter in unit order and
+// streams their tiles through the ring without a break; a 16-byte record per
+// stage tells the consumers which item a tile belongs to and whether it is
+// the item's first or last. A consumer epilogue (warp merge, output or
+// partial, arrival, combine) overlaps the loads of the next item.
+
+struct StageInfo {
+  int item;   // work item, or -1: no more work
+  int rows;   // valid keys in the tile
+  int first;  // first tile of the item
+  int last;   // last tile of the item
+};
+
+struct ItemCoord {
+  int b, g, unit, split, hsl, h0, nh;
+};
+
+__device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item) {
+  ItemCoord c;
+  c.hsl = item % p.hslices;
+  const int rest = item / p.hslices;
+  c.split = rest % p.nsplit;
+  c.unit = rest / p.nsplit;
+  c.b = c.unit / p.K;
+  c.g = c.unit % p.K;
+  c.h0 = c.g * p.G + c.hsl * kDecHeadsPerCta;
+  c.nh = min(kDecHeadsPerCta, p.G - c.hsl * kDecHeadsPerCta);
+  return c;
 }
 
-// ---------------------------------------------------------------------------
-// bf16 tensor-core decode
+// End of a work item: merge the four warps, then write the output (a unit
+// with a single split) or the split's partial for decode_combine_kernel.
+template <int D>
+__device__ __forceinline__ void item_epilogue(const DecodeParams& p, const ItemCoord& c, const WarpState<D>& st,
+                                              float* merge, int tid, int warp, int lane) {
+  __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(p.out) + ((size_t)c.b * p.H + c.h0) * D;
+  const int len = valid_len(__ldg(p.seqlens + c.b), p.S_max);
+  const int ns = (len + p.chunk - 1) / p.chunk;  // splits that hold keys of this unit
+  consumer_bar();  // the previous epilogue has finished with the scratch
+  stash_warp_state<D>(merge, st, warp, lane);
+  consumer_bar();
+  const size_t part = ((size_t)c.unit * p.nsplit + c.split) * p.G + (size_t)c.hsl * kDecHeadsPerCta;
+  for (int i = tid; i < c.nh * D; i += kDecConsumerWarps * 32) {
+    const int h = i / D, dim = i % D;
+    float M, L, O;
+    merged<D>(merge, h, dim, M, L, O);
+    if (ns == 1) {
+      out_row[i] = __float2bfloat16_rn(O / L);
+    } else {
+      p.ws_o[(part + h) * D + dim] = O;
+      if (dim == 0) p.ws_ml[part + h] = make_float2(M, L);
+    }
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const DecodeParams p) {
   using C = DecCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  float* merge = reinterpret_cast<float*>(smem + C::kMergeOff);
+  StageInfo* info = reinterpret_cast<StageInfo*>(smem + C::kInfoOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* empty = full + C::kStages;
-
-  const DecItem w = decode_item(p, kDecHeadsPerCta);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
 
-  if (w.t_begin >= w.t_end) {
-    // No key of this sequence falls in this split. With a single split this
-    // CTA owns the output (len_b == 0 -> zeros); otherwise the combine only
-    // reads the first ceil(len_b / chunk) splits.
-    if (p.nsplit == 1)
-      for (int i = threadIdx.x; i < w.nh * D; i += blockDim.x)
-        out[((size_t)w.b * p.H + w.h0 + i / D) * D + (i % D)] = __float2bfloat16_rn(0.f);
+  if (smem_u32(smem) & 1023u) {  // the swizzle pattern needs 1024-byte aligned stages
+    if (threadIdx.x == 0) raise_error(GQA_DEVERR_TIMEOUT);
     return;
   }
-  const int ntiles = (w.t_end - w.t_begin + kDecTileKeys - 1) / kDecTileKeys;
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -136,6 +414,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     fence_mbar_init();
   }
   __syncthreads();
+  // the combine kernel may be scheduled now; it waits for this grid to finish
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == kDecConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -143,191 +423,74 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
       const uint64_t policy = l2_policy_evict_first();
-      const int row_base = w.unit * p.S_max;
-      int issued = 0;
-      for (int it = 0; it < ntiles; ++it) {
-        const int s = it % C::kStages;
-        if (it >= C::kStages && !mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1)) break;
-        const int t0 = w.t_begin + it * kDecTileKeys;
-        const int rows = min(kDecTileKeys, w.t_end - t0);
-        const int nbox = (rows + kDecBoxRows - 1) / kDecBoxRows;
-        uint8_t* ks = smem + s * C::kStageBytes;
-        uint8_t* vs = ks + C::kTileBytes;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(nbox * kDecBoxRows * 128 * C::kHalves * 2));
-        for (int bx = 0; bx < nbox; ++bx) {
-#pragma unroll
-          for (int hf = 0; hf < C::kHalves; ++hf) {
-            const int off = hf * C::kHalfBytes + bx * kDecBoxRows * 128;
-            tma_load_2d(ks + off, &tm_k, hf * 64, row_base + t0 + bx * kDecBoxRows, &full[s], policy);
-            tma_load_2d(vs + off, &tm_v, hf * 64, row_base + t0 + bx * kDecBoxRows, &full[s], policy);
+      int it = 0;  // ring position
+      bool ok = true;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+      for (;;) {
+        const int item = take_ticket(p.ws_queue, p.tag) - 1;
+        if (item < 0 || item >= p.nitems) break;
+        const ItemCoord c = item_coord(p, item);
+        const int raw = __ldg(p.seqlens + c.b);
+        const int len = valid_len(raw, p.S_max);
+        if (len != raw && c.g == 0 && c.split == 0 && c.hsl == 0) raise_error(GQA_DEVERR_SEQLEN);
+        const int t_begin = c.split * p.chunk;
+        const int t_end = min(len, t_begin + p.chunk);
+        if (t_begin >= t_end) {
+          if (c.split == 0) {  // an empty sequence: zeros for this item's heads
+            uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)c.b * p.H + c.h0) * D);
+            for (int i = 0; i < c.nh * D / 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
           }
+          continue;
         }
-        ++issued;
+        const int ntiles = (t_end - t_begin + kDecTileKeys - 1) / kDecTileKeys;
+        const int row_base = c.unit * p.S_max;
+        for (int tt = 0; tt < ntiles && ok; ++tt, ++it) {
+          const int s = it % C::kStages;
+          if (it >= C::kStages) ok = mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1);
+          if (!ok) break;
+          const int t0 = t_begin + tt * kDecTileKeys;
+          const int rows = min(kDecTileKeys, t_end - t0);
+          info[s] = StageInfo{item, rows, tt == 0, tt == ntiles - 1};
+          issue_tile<D>(smem + s * C::kStageBytes, &full[s], &tm_k, &tm_v, row_base + t0, rows, policy);
+        }
+        if (!ok) break;
       }
-      // Wait for this CTA's own loads to land before the block may exit.
-      for (int it = max(0, issued - C::kStages); it < issued; ++it)
-        mbar_wait_bounded(&full[it % C::kStages], (it / C::kStages) & 1);
+      // no more work: a record without loads ends the consumers' loop
+      if (ok) {
+        const int s = it % C::kStages;
+        if (it >= C::kStages) ok = mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1);
+        if (ok) {
+          info[s] = StageInfo{-1, 0, 0, 0};
+          mbar_arrive(&full[s]);
+          ++it;
+        }
+      }
+      // this CTA's own loads must land before the block may exit
+      for (int j = max(0, it - C::kStages); j < it; ++j) mbar_wait_bounded(&full[j % C::kStages], (j / C::kStages) & 1);
     }
     return;
   }
 
   // -------------------------------------------------------------- consumers
-  // Q^T as the B operand (k = dims, n = heads): lane holds head lane/4,
-  // dims 2*(lane%4) + {0,1} (b0) and + 8 (b1) of every 16-dim step.
+  const int tid = threadIdx.x;  // 0..127
+  const int kb = warp * 16;
   uint32_t qf[D / 16][2];
-  {
-    const int hn = lane >> 2;
-    const bool hv = hn < w.nh;
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(p.q) +
-                                                             ((size_t)w.b * p.H + w.h0 + (hv ? hn : 0)) * D);
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const uint32_t lo = __ldg(qrow + ks * 8 + (lane & 3));
-      const uint32_t hi = __ldg(qrow + ks * 8 + 4 + (lane & 3));
-      qf[ks][0] = hv ? lo : 0u;
-      qf[ks][1] = hv ? hi : 0u;
-    }
-  }
-
-  // Running state for heads a = 2*(lane%4) and b = a + 1 (log2 units).
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-  float o[D / 16][4];
-#pragma unroll
-  for (int md = 0; md < D / 16; ++md) o[md][0] = o[md][1] = o[md][2] = o[md][3] = 0.f;
-
-  const int kb = warp * 16;  // this warp's 16 keys inside every tile
-  // ldmatrix row/column assignment (lane -> 8x8 matrix lane/8)
-  const int k_row = kb + (lane & 7) + ((lane >> 3) & 1) * 8;  // K: matrices (r0-7,c0-7) (r8-15,c0-7) (r0-7,c8-15) ...
-  const int k_col8 = (lane >> 4);
-  const int v_row = kb + (lane & 7) + (lane >> 4) * 8;  // V^T: matrices (d0-7,k0-7) (d8-15,k0-7) (d0-7,k8-15) ...
-  const int v_col8 = (lane >> 3) & 1;
-
-  for (int it = 0; it < ntiles; ++it) {
+  WarpState<D> st;
+  ItemCoord cur{};
+  for (int it = 0;; ++it) {
     const int s = it % C::kStages;
-    if (!mbar_wait_bounded(&full[s], (it / C::kStages) & 1)) break;
-    const int t0 = w.t_begin + it * kDecTileKeys;
-    const int rows = min(kDecTileKeys, w.t_end - t0);
-    if (kb < rows) {
-      const uint32_t k_base = smem_u32(smem + s * C::kStageBytes);
-      const uint32_t v_base = k_base + C::kTileBytes;
-
-      // S^T = K * Q^T
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const int chunk = ks * 2 + k_col8;  // 16-byte chunk index along the row
-        const uint32_t addr = k_base + (chunk >> 3) * C::kHalfBytes + sw128(k_row, chunk & 7);
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4(addr, a0, a1, a2, a3);
-        mma_bf16_16816(c, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
-      }
-
-      // online softmax over this block's keys (key kb + lane/4 in c0/c1, +8 in c2/c3)
-      const int key0 = kb + (lane >> 2);
-      const bool v0 = key0 < rows, v1 = key0 + 8 < rows;
-      const float x0 = v0 ? c[0] * p.scale_log2 : -INFINITY;
-      const float x1 = v0 ? c[1] * p.scale_log2 : -INFINITY;
-      const float x2 = v1 ? c[2] * p.scale_log2 : -INFINITY;
-      const float x3 = v1 ? c[3] * p.scale_log2 : -INFINITY;
-      float mx_a = fmaxf(x0, x2), mx_b = fmaxf(x1, x3);
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
-        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
-      }
-      const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-      const float al_a = fast_exp2(m_a - mn_a), al_b = fast_exp2(m_b - mn_b);
-      m_a = mn_a;
-      m_b = mn_b;
-      const float p0 = fast_exp2(x0 - mn_a), p1 = fast_exp2(x1 - mn_b);
-      const float p2 = fast_exp2(x2 - mn_a), p3 = fast_exp2(x3 - mn_b);
-      l_a = l_a * al_a + p0 + p2;
-      l_b = l_b * al_b + p1 + p3;
-#pragma unroll
-      for (int md = 0; md < D / 16; ++md) {
-        o[md][0] *= al_a;
-        o[md][1] *= al_b;
-        o[md][2] *= al_a;
-        o[md][3] *= al_b;
-      }
-
-      // P^T (k = keys, n = heads) from the S^T accumulator layout
-      const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
-      const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
-
-      // keys of this block past the end of the sequence: zero their V^T
-      // entries (the rows may hold anything, NaN included)
-      uint32_t mask_lo = 0xffffffffu, mask_hi = 0xffffffffu;
-      if (kb + 16 > rows) {
-        const int lim = rows - kb;
-        const int kk = 2 * (lane & 3);
-        mask_lo = (kk < lim ? 0x0000ffffu : 0u) | (kk + 1 < lim ? 0xffff0000u : 0u);
-        mask_hi = (kk + 8 < lim ? 0x0000ffffu : 0u) | (kk + 9 < lim ? 0xffff0000u : 0u);
-      }
-
-      // O^T += V^T * P^T
-#pragma unroll
-      for (int md = 0; md < D / 16; ++md) {
-        const int chunk = md * 2 + v_col8;
-        const uint32_t addr = v_base + (chunk >> 3) * C::kHalfBytes + sw128(v_row, chunk & 7);
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4_trans(addr, a0, a1, a2, a3);
-        mma_bf16_16816(o[md], a0 & mask_lo, a1 & mask_lo, a2 & mask_hi, a3 & mask_hi, pb0, pb1);
-      }
+    if (!mbar_wait_bounded(&full[s], (it / C::kStages) & 1)) break;  // every consumer warp sees the same barrier
+    const StageInfo si = info[s];
+    if (si.item < 0) break;
+    if (si.first) {
+      cur = item_coord(p, si.item);
+      load_q_frag<D>(qf, static_cast<const __nv_bfloat16*>(p.q) + ((size_t)cur.b * p.H + cur.h0) * D, lane, cur.nh);
+      st.reset();
     }
+    if (kb < si.rows) warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-  }
-
-  // ---------------------------------------------------------------- merge
-#pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, off);
-    l_b += __shfl_xor_sync(0xffffffffu, l_b, off);
-  }
-  float* red_m = reinterpret_cast<float*>(smem);                  // [4][8]
-  float* red_l = red_m + kDecConsumerWarps * kDecHeadsPerCta;     // [4][8]
-  float* red_o = red_l + kDecConsumerWarps * kDecHeadsPerCta;     // [4][8][D]
-  asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumerWarps * 32) : "memory");  // stage buffers now free
-  {
-    const int ha = 2 * (lane & 3);
-    if (lane < 4) {
-      red_m[warp * 8 + ha] = m_a;
-      red_m[warp * 8 + ha + 1] = m_b;
-      red_l[warp * 8 + ha] = l_a;
-      red_l[warp * 8 + ha + 1] = l_b;
-    }
-    float* ow = red_o + warp * kDecHeadsPerCta * D;
-    const int dr = lane >> 2;
-#pragma unroll
-    for (int md = 0; md < D / 16; ++md) {
-      ow[ha * D + md * 16 + dr] = o[md][0];
-      ow[(ha + 1) * D + md * 16 + dr] = o[md][1];
-      ow[ha * D + md * 16 + dr + 8] = o[md][2];
-      ow[(ha + 1) * D + md * 16 + dr + 8] = o[md][3];
-    }
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumerWarps * 32) : "memory");
-
-  const size_t part = ((size_t)w.unit * p.nsplit + w.split) * p.G + (size_t)w.hsl * kDecHeadsPerCta;
-  for (int i = threadIdx.x; i < w.nh * D; i += kDecConsumerWarps * 32) {
-    const int h = i / D, dim = i % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int ww = 0; ww < kDecConsumerWarps; ++ww) M = fmaxf(M, red_m[ww * 8 + h]);
-    float L = 0.f, O = 0.f;
-#pragma unroll
-    for (int ww = 0; ww < kDecConsumerWarps; ++ww) {
-      const float f = fast_exp2(red_m[ww * 8 + h] - M);
-      L += red_l[ww * 8 + h] * f;
-      O += red_o[(ww * kDecHeadsPerCta + h) * D + dim] * f;
-    }
-    if (p.nsplit == 1) {
-      out[((size_t)w.b * p.H + w.h0 + h) * D + dim] = __float2bfloat16_rn(O / L);
-    } else {
-      p.ws_o[(part + h) * D + dim] = O;
-      if (dim == 0) p.ws_ml[part + h] = make_float2(M, L);
-    }
+    if (si.last) item_epilogue<D>(p, cur, st, merge, tid, warp, lane);
   }
 }
 
@@ -426,48 +589,103 @@ __global__ void __launch_bounds__(kDecF32Threads) decode_f32_kernel(const float*
 }
 
 // ---------------------------------------------------------------------------
-// Split-KV combine: out[b,h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,
-// M = max_s m_s, over the ceil(len_b / chunk) splits that hold keys.
-// One CTA of D threads per (b, h).
+// Split-KV combine (the log-sum-exp merge of the partials):
+//   M = max_s m_s,  out[b,h] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s
+// over the ns = ceil(len_b / chunk) splits that hold keys (units with one
+// split were finished by the decode kernel). One CTA of 128 threads per
+// (b, h): four groups of 32 threads take every fourth split, each thread one
+// 16-byte column group, eight loads in flight; the groups are summed in
+// shared memory. Launched as a programmatic dependent of the decode kernel:
+// it waits for that grid before reading the partials.
 
-template <typename OutT>
-__global__ void decode_combine_kernel(OutT* __restrict__ out, const float* __restrict__ ws_o,
-                                      const float2* __restrict__ ws_ml, const int32_t* __restrict__ seqlens, int H,
-                                      int K, int S_max, int G, int chunk, int nsplit, int D) {
+constexpr int kCombThreads = 128;
+
+template <typename OutT, int D>
+__global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(OutT* __restrict__ out,
+                                                                     const float* __restrict__ ws_o,
+                                                                     const float2* __restrict__ ws_ml,
+                                                                     const int32_t* __restrict__ seqlens, int H, int K,
+                                                                     int S_max, int G, int chunk, int nsplit,
+                                                                     int skip_single) {
+  __shared__ float sw[kMaxCombineSplits];
+  __shared__ float4 sacc[4][D / 4];
+  __shared__ float sred[2];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
   const int g = h / G, j = h % G;
-  int len = __ldg(seqlens + b);
-  if (len < 0 || len > S_max) len = 0;
+  const int len = valid_len(__ldg(seqlens + b), S_max);
   const int ns = (len + chunk - 1) / chunk;
+  const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
+  if (ns == 0) {  // empty sequence
+    for (int i = tid; i < D; i += kCombThreads) store_out<OutT>(out + (size_t)bh * D + i, 0.f);
+    return;
+  }
+  if (ns == 1 && skip_single) return;
   const size_t base = ((size_t)(b * K + g) * nsplit) * G + j;  // split s at base + s*G
-  const int dim = threadIdx.x;
+  // max and weights
   float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, __ldg(&ws_ml[base + (size_t)s * G].x));
-  float L = 0.f, acc = 0.f;
-  int s = 0;
-  for (; s + 4 <= ns; s += 4) {
-    float2 ml[4];
-    float ov[4];
+  for (int s = tid; s < ns; s += kCombThreads) M = fmaxf(M, __ldcg(&ws_ml[base + (size_t)s * G].x));
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      ml[u] = __ldg(&ws_ml[base + (size_t)(s + u) * G]);
-      ov[u] = __ldg(&ws_o[(base + (size_t)(s + u) * G) * D + dim]);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float f = fast_exp2(ml[u].x - M);
-      L += ml[u].y * f;
-      acc += ov[u] * f;
-    }
-  }
-  for (; s < ns; ++s) {
-    const float2 ml = __ldg(&ws_ml[base + (size_t)s * G]);
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (lane == 0) sw[grp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(sw[0], sw[1]), fmaxf(sw[2], sw[3]));
+  __syncthreads();
+  float L = 0.f;
+  for (int s = tid; s < ns; s += kCombThreads) {
+    const float2 ml = __ldcg(&ws_ml[base + (size_t)s * G]);
     const float f = fast_exp2(ml.x - M);
+    sw[s] = f;
     L += ml.y * f;
-    acc += __ldg(&ws_o[(base + (size_t)s * G) * D + dim]) * f;
   }
-  store_out<OutT>(out + (size_t)bh * D + dim, ns > 0 ? acc / L : 0.f);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  if (lane == 0) sacc[grp][0].x = L;
+  __syncthreads();
+  if (tid == 0) sred[0] = sacc[0][0].x + sacc[1][0].x + sacc[2][0].x + sacc[3][0].x;
+  __syncthreads();
+  // weighted sum of the partial O rows
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane < D / 4) {
+    constexpr int kBatch = 8;
+    for (int s0 = grp; s0 < ns; s0 += 4 * kBatch) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int s = s0 + 4 * u;
+        v[u] = s < ns ? __ldcg(reinterpret_cast<const float4*>(ws_o + (base + (size_t)s * G) * D) + lane)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int s = s0 + 4 * u;
+        const float f = s < ns ? sw[s] : 0.f;
+        acc.x += v[u].x * f;
+        acc.y += v[u].y * f;
+        acc.z += v[u].z * f;
+        acc.w += v[u].w * f;
+      }
+    }
+    sacc[grp][lane] = acc;
+  }
+  __syncthreads();
+  if (tid < D / 4) {
+    const float inv = 1.f / sred[0];
+    float4 t = sacc[0][tid];
+#pragma unroll
+    for (int q = 1; q < 4; ++q) {
+      t.x += sacc[q][tid].x;
+      t.y += sacc[q][tid].y;
+      t.z += sacc[q][tid].z;
+      t.w += sacc[q][tid].w;
+    }
+    OutT* o = out + (size_t)bh * D + tid * 4;
+    store_out<OutT>(o + 0, t.x * inv);
+    store_out<OutT>(o + 1, t.y * inv);
+    store_out<OutT>(o + 2, t.z * inv);
+    store_out<OutT>(o + 3, t.w * inv);
+  }
 }
 
 }  // namespace gqa

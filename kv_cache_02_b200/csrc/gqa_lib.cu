@@ -8,9 +8,12 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <random>
 
 #include "../../include/gqa.h"
 #include "append_meanpool.cuh"
@@ -83,12 +86,28 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ER
 // decode launch plan
 
 struct DecodePlan {
-  int chunk = 0;    // keys per split (multiple of 64)
-  int nsplit = 1;   // splits per (b, g)
-  int hslices = 1;  // head slices per (b, g)
-  long long grid = 0;
+  int chunk = 0;       // keys per split (multiple of 64)
+  int nsplit = 1;      // splits per (b, g)
+  int hslices = 1;     // head slices per (b, g)
+  long long grid = 0;  // bf16: persistent CTAs; f32: one CTA per work item
   size_t ws_bytes = 0;
+  size_t ws_ml_off = 0, ws_queue_off = 0;
 };
+
+// A 40-bit tag that differs on every decode call of this process and, being
+// seeded at random, from the tags of other processes: a work counter left by
+// an earlier call (or uninitialised memory) does not match it.
+unsigned long long next_call_tag() {
+  static std::atomic<unsigned long long> counter{0};
+  static unsigned long long seed = [] {
+    std::random_device rd;
+    const unsigned long long t =
+        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+    return ((((unsigned long long)rd()) << 32) ^ rd() ^ (t * 0x9E3779B97F4A7C15ull)) | 1ull;
+  }();
+  const unsigned long long t = (seed + 2ull * counter.fetch_add(1)) & ((1ull << 40) - 1);
+  return t ? t : 1ull;
+}
 
 bool valid_decode_shape(int B, int H, int K, int S_max, int d) {
   if (B < 0 || H <= 0 || K <= 0 || S_max <= 0) return false;
@@ -99,18 +118,39 @@ bool valid_decode_shape(int B, int H, int K, int S_max, int d) {
   return true;
 }
 
+// Resident persistent decode CTAs per SM for head dim D (2 on B200), cached per device.
+template <int D>
+int decode_ctas_per_sm(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return 2;
+  if (cache[dev] == 0) {
+    int n = 0;
+    using C = gqa::DecCfg<D>;
+    if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_bf16_kernel<D>, gqa::kDecThreads,
+                                                      C::kSmemBytes) != cudaSuccess ||
+        n <= 0) {
+      cudaGetLastError();  // no GPU here: plan with the B200 figure
+      n = 2;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gqa_dtype dt, int sms) {
   DecodePlan pl;
   const int G = H / K;
   const int heads_per_cta = dt == GQA_BF16 ? gqa::kDecHeadsPerCta : gqa::kDecF32HeadsPerCta;
   pl.hslices = (G + heads_per_cta - 1) / heads_per_cta;
   const long long units = (long long)B * K * pl.hslices;
-  const int max_splits = (S_max + 63) / 64;
+  const int max_splits = std::min((S_max + 63) / 64, gqa::kMaxCombineSplits);
   int splits;
   if (num_splits > 0) {
     splits = std::min(num_splits, max_splits);
   } else {
-    // about four waves of two CTAs per SM, never below 256 keys per split
+    // about eight work items per SM, never below 256 keys per split
     const long long target = 8ll * sms;
     splits = (int)std::max<long long>(1, (target + units - 1) / std::max<long long>(units, 1));
     splits = std::min(splits, std::max(1, (S_max + 255) / 256));
@@ -120,11 +160,25 @@ DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gq
   chunk = (chunk + 63) / 64 * 64;
   pl.chunk = chunk;
   pl.nsplit = (S_max + chunk - 1) / chunk;
-  pl.grid = (long long)B * K * pl.nsplit * pl.hslices;
-  if (pl.nsplit > 1) {
-    const size_t parts = (size_t)B * K * pl.nsplit * G;
-    pl.ws_bytes = parts * d * sizeof(float) + parts * sizeof(float2);
+  const size_t parts = (size_t)B * K * pl.nsplit * G;
+  const size_t part_bytes = pl.nsplit > 1 ? parts * d * sizeof(float) + parts * sizeof(float2) : 0;
+  pl.ws_ml_off = parts * d * sizeof(float);
+  if (dt == GQA_BF16) {
+    // persistent CTAs that take work items from a counter in the workspace
+    const int dev = current_device();
+    const int per_sm = d == 128 ? decode_ctas_per_sm<128>(dev) : decode_ctas_per_sm<64>(dev);
+    const long long items = units * pl.nsplit;
+    pl.grid = std::max<long long>(1, std::min<long long>(items, (long long)per_sm * sms));
+    if (items + pl.grid >= (1ll << 24)) {  // beyond the work counter
+      pl.ws_bytes = (size_t)-1;
+      return pl;
+    }
+    pl.ws_queue_off = (part_bytes + 15) / 16 * 16;
+    pl.ws_bytes = pl.ws_queue_off + 16;
+    return pl;
   }
+  pl.grid = units * pl.nsplit;
+  pl.ws_bytes = part_bytes;
   return pl;
 }
 
@@ -136,14 +190,7 @@ int launch_decode_bf16(const DecodePlan& pl, const DecodeParams& p, const void* 
   if (!encode_rows_bf16(&tk, kc, rows, D, gqa::kDecBoxRows) || !encode_rows_bf16(&tv, vc, rows, D, gqa::kDecBoxRows))
     return GQA_ERR_CUDA;
   using C = gqa::DecCfg<D>;
-  static int configured[kMaxDevices] = {0};
-  const int dev = current_device();
-  if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
-    if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      return GQA_ERR_CUDA;
-    configured[dev] = 1;
-  }
+  decode_ctas_per_sm<D>(current_device());  // sets the shared-memory attribute once per device
   gqa::decode_bf16_kernel<D><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(tk, tv, p);
   return launch_status();
 }
@@ -230,6 +277,7 @@ size_t gqa_decode_workspace_bytes(int B, int H, int K, int S_max, int d, int num
   // which does not change the workspace size; take the larger of the two
   const DecodePlan a = plan_decode(B, H, K, S_max, d, num_splits, GQA_BF16, sm_count(dev));
   const DecodePlan b = plan_decode(B, H, K, S_max, d, num_splits, GQA_F32, sm_count(dev));
+  if (a.ws_bytes == (size_t)-1) return 0;
   return std::max(a.ws_bytes, b.ws_bytes);
 }
 
@@ -244,18 +292,23 @@ int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cach
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return GQA_ERR_ALIGN;
   const int dev = current_device();
   const DecodePlan pl = plan_decode(B, H, K, S_max, d, num_splits, dtype, sm_count(dev));
+  if (pl.ws_bytes == (size_t)-1) return GQA_ERR_SHAPE;  // more work items than the work counter holds
   if (pl.ws_bytes > 0) {
     if (!workspace || workspace_bytes < pl.ws_bytes) return GQA_ERR_INVALID_ARG;
     if (!aligned16(workspace)) return GQA_ERR_ALIGN;
   }
   const int G = H / K;
+  cudaStream_t st = (cudaStream_t)stream;
   DecodeParams p;
   p.q = q;
   p.out = out;
   p.ws_o = static_cast<float*>(workspace);
-  p.ws_ml = pl.ws_bytes ? reinterpret_cast<float2*>(static_cast<char*>(workspace) +
-                                                    (size_t)B * K * pl.nsplit * G * d * sizeof(float))
-                        : nullptr;
+  p.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + pl.ws_ml_off);
+  p.ws_queue = dtype == GQA_BF16 ? reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) +
+                                                                         pl.ws_queue_off)
+                                 : nullptr;
+  p.nitems = (int)((long long)B * K * pl.hslices * pl.nsplit);
+  p.tag = next_call_tag();
   p.seqlens = seqlens;
   p.B = B;
   p.H = H;
@@ -266,7 +319,6 @@ int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cach
   p.chunk = pl.chunk;
   p.nsplit = pl.nsplit;
   p.scale_log2 = scale * 1.4426950408889634f;
-  cudaStream_t st = (cudaStream_t)stream;
   int rc;
   if (dtype == GQA_BF16)
     rc = d == 128 ? launch_decode_bf16<128>(pl, p, k_cache, v_cache, B, K, S_max, st)
@@ -275,12 +327,37 @@ int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cach
     rc = d == 128 ? launch_decode_f32<128>(pl, p, k_cache, v_cache, st)
                   : launch_decode_f32<64>(pl, p, k_cache, v_cache, st);
   if (rc != GQA_OK || pl.nsplit == 1) return rc;
+  // the split-KV combine, as a programmatic dependent launch: its launch
+  // overlaps the decode kernel, and it waits for that grid before reading
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long long)B * H));
+  cfg.blockDim = dim3(gqa::kCombThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  const int skip_single = dtype == GQA_BF16 ? 1 : 0;  // bf16 units with one split are already written
   if (dtype == GQA_BF16)
-    gqa::decode_combine_kernel<__nv_bfloat16><<<(unsigned)((long long)B * H), d, 0, st>>>(
-        static_cast<__nv_bfloat16*>(out), p.ws_o, p.ws_ml, seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, d);
+    e = d == 128 ? cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<__nv_bfloat16, 128>,
+                                      static_cast<__nv_bfloat16*>(out), (const float*)p.ws_o, (const float2*)p.ws_ml,
+                                      seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single)
+                 : cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<__nv_bfloat16, 64>,
+                                      static_cast<__nv_bfloat16*>(out), (const float*)p.ws_o, (const float2*)p.ws_ml,
+                                      seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single);
   else
-    gqa::decode_combine_kernel<float><<<(unsigned)((long long)B * H), d, 0, st>>>(
-        static_cast<float*>(out), p.ws_o, p.ws_ml, seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, d);
+    e = d == 128 ? cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<float, 128>, static_cast<float*>(out),
+                                      (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, H, K, S_max, G, pl.chunk,
+                                      pl.nsplit, skip_single)
+                 : cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<float, 64>, static_cast<float*>(out),
+                                      (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, H, K, S_max, G, pl.chunk,
+                                      pl.nsplit, skip_single);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
+  }
   return launch_status();
 }
 

@@ -145,3 +145,43 @@ def test_decode_full_size_sampled(gqa, name):
     sel = np.concatenate([sel, [[0, 0], [w.B - 1, w.H - 1]]]).astype(np.int32)
     ref = oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], scale, sel=sel)
     assert_close(got[sel[:, 0], sel[:, 1]], ref, name)
+
+
+# ---------------------------------------------------------------------------
+# automatic splits: many splits per unit, and the in-kernel combine by the
+# last split to arrive
+
+AUTO = [
+    # B, H, K, d, S_max, lens
+    (1, 8, 1, 128, 65536, (65536,)),                                  # one unit, a wide combine
+    (37, 16, 2, 128, 700, tuple(int(x) for x in np.random.default_rng(3).integers(0, 701, 37))),
+    (64, 8, 8, 64, 130, (1, 63, 64, 65, 127, 128, 129, 130) * 8),     # tile-edge lengths, many small units
+    (3, 64, 1, 128, 9000, (9000, 4097, 1)),                           # MQA: eight head slices per unit
+]
+
+
+@pytest.mark.parametrize("shape", AUTO, ids=lambda s: f"B{s[0]}H{s[1]}K{s[2]}d{s[3]}S{s[4]}")
+def test_decode_auto_splits(gqa, shape):
+    B, H, K, d, S_max, lens = shape
+    inp = make(B, H, K, d, S_max, lens, synth.BF16, 0x57A0 + B + H)
+    scale = 1.0 / np.sqrt(d)
+    got, status = run_decode(gqa, inp, scale, 0)
+    assert status == (0, 0)
+    ref = oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], scale)
+    assert_close(got, ref, str(shape[:5]))
+
+
+def test_decode_workspace_needs_no_initialisation(gqa):
+    inp = make(4, 32, 8, 128, 3000, (3000, 2999, 1, 1500), synth.BF16, 0x57B0)
+    B, H, d = inp["q"].shape
+    q, kc, vc = dev(inp["q"]), dev(inp["k_cache"]), dev(inp["v_cache"])
+    lens = dev(inp["seqlens"])
+    ws_bytes = gqa.gqa_decode_workspace_bytes(B, H, 8, 3000, d, 0)
+    ref = oracle.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["seqlens"], 0.1)
+    for fill in (0xFF, 0x00, 0xA5):
+        ws = torch.full((ws_bytes,), fill, dtype=torch.uint8, device="cuda")
+        for _ in range(2):  # the same workspace twice in a row
+            out = torch.empty_like(q)
+            gqa.gqa_decode(out, q, kc, vc, lens, 0.1, 0, ws)
+            assert gqa.gqa_get_last_error() == (0, 0)
+            assert_close(host(out), ref, f"fill {fill:#x}")
