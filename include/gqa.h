@@ -125,6 +125,28 @@ GQA_API int gqa_decode(void* out, const void* q, const void* k_cache, const void
                gqa_dtype dtype, gqa_stream_t stream);
 
 /*
+ * gqa_decode_append - one decode step with the new token's append fused in:
+ * the effect of gqa_kv_append(k_cache, v_cache, k_new, v_new, pos, ...)
+ * followed by gqa_decode(..., seqlens = pos + 1, ...), in one pass over the
+ * cache ("GQA 完全拆解", section 解码推理的内存账本: the new query attends to
+ * every cached key including its own, and the new K, V row joins the cache).
+ *
+ * k_cache, v_cache : [B, K, S_max, d]; row pos[b] of every (b, g) is written.
+ * k_new, v_new     : [B, K, d], the new token's K and V.
+ * pos              : [B] int32, device: the length of each sequence before
+ *                    the append. pos[b] outside [0, S_max) sets
+ *                    GQA_DEVERR_APPEND_POS, writes nothing and gives
+ *                    out[b] = 0.
+ * Everything else as for gqa_decode; the workspace size is
+ * gqa_decode_workspace_bytes of the same shape. bf16 runs as one decode
+ * kernel (plus the split combine); f32 launches the append first.
+ */
+GQA_API int gqa_decode_append(void* out, const void* q, void* k_cache, void* v_cache, const void* k_new,
+                              const void* v_new, const int32_t* pos, int B, int H, int K, int S_max, int d,
+                              float scale, int num_splits, void* workspace, size_t workspace_bytes, gqa_dtype dtype,
+                              gqa_stream_t stream);
+
+/*
  * gqa_decode_noalloc - gqa_decode without a caller-supplied workspace.
  *
  * The paper has no counterpart to this call. It is for callers that cannot

@@ -63,6 +63,12 @@ struct DecodeParams {
   void* out;
   float* ws_o;                 // [B*K*nsplit*G, D] partial O (unnormalised, relative to m)
   float2* ws_ml;               // [B*K*nsplit*G] partial (m, l), m in log2 units
+  // fused append (gqa_decode_append): seqlens holds pos, lengths are pos + len_add
+  const void* k_new;           // [B, K, D] or null
+  const void* v_new;
+  void* k_cache_w;             // the caches, written at row pos[b]
+  void* v_cache_w;
+  int len_add;                 // 0 (decode) or 1 (decode after append)
   unsigned long long* ws_queue;  // work-item counter of the persistent kernel: tag | count
   int nitems;                  // B * K * nsplit * hslices
   const int32_t* seqlens;
@@ -319,7 +325,7 @@ __device__ __forceinline__ DecItem decode_item(const DecodeParams& p, int heads_
   it.unit = rest / p.nsplit;
   it.b = it.unit / p.K;
   it.g = it.unit % p.K;
-  int len = __ldg(p.seqlens + it.b);
+  int len = __ldg(p.seqlens + it.b) + p.len_add;
   if (len < 0 || len > p.S_max) {
     if (it.split == 0 && it.hsl == 0 && it.g == 0 && threadIdx.x == 0) raise_error(GQA_DEVERR_SEQLEN);
     len = 0;
@@ -341,10 +347,10 @@ __device__ __forceinline__ DecItem decode_item(const DecodeParams& p, int heads_
 // partial, arrival, combine) overlaps the loads of the next item.
 
 struct StageInfo {
-  int item;   // work item, or -1: no more work
-  int rows;   // valid keys in the tile
-  int first;  // first tile of the item
-  int last;   // last tile of the item
+  int item;     // work item, or -1: no more work
+  int rows;     // valid keys in the tile
+  int flags;    // 1: first tile of the item, 2: last tile of the item
+  int new_row;  // row of the tile that holds the appended token, or -1
 };
 
 struct ItemCoord {
@@ -370,7 +376,7 @@ template <int D>
 __device__ __forceinline__ void item_epilogue(const DecodeParams& p, const ItemCoord& c, const WarpState<D>& st,
                                               float* merge, int tid, int warp, int lane) {
   __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(p.out) + ((size_t)c.b * p.H + c.h0) * D;
-  const int len = valid_len(__ldg(p.seqlens + c.b), p.S_max);
+  const int len = valid_len(__ldg(p.seqlens + c.b) + p.len_add, p.S_max);
   const int ns = (len + p.chunk - 1) / p.chunk;  // splits that hold keys of this unit
   consumer_bar();  // the previous epilogue has finished with the scratch
   stash_warp_state<D>(merge, st, warp, lane);
@@ -387,6 +393,34 @@ __device__ __forceinline__ void item_epilogue(const DecodeParams& p, const ItemC
       if (dim == 0) p.ws_ml[part + h] = make_float2(M, L);
     }
   }
+}
+
+// The appended token (gqa_decode_append): its K and V replace row `r` of the
+// tile just landed in shared memory (one warp, one 16-byte chunk per lane)
+// and are written to the cache at that row. The tile's rows are cache rows
+// t0 .. t0+rows-1, so row r is cache row len-1 = pos.
+template <int D>
+__device__ __forceinline__ void append_row(const DecodeParams& p, const ItemCoord& c, uint8_t* stage, int r,
+                                           int lane) {
+  using C = DecCfg<D>;
+  constexpr int kChunks = D / 8;  // 16-byte chunks per row
+  const int pos = __ldg(p.seqlens + c.b);
+  if (lane < 2 * kChunks) {
+    const bool is_v = lane >= kChunks;
+    const int ch = is_v ? lane - kChunks : lane;
+    const size_t row = (size_t)c.b * p.K + c.g;  // unit (b, g)
+    const uint4 val = __ldg(reinterpret_cast<const uint4*>(
+                                static_cast<const __nv_bfloat16*>(is_v ? p.v_new : p.k_new) + row * D) + ch);
+    uint8_t* dst = stage + (is_v ? C::kTileBytes : 0) + (ch >> 3) * C::kHalfBytes + sw128((uint32_t)r, ch & 7);
+    *reinterpret_cast<uint4*>(dst) = val;
+    if (c.hsl == 0) {  // one head slice writes the cache
+      __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(is_v ? p.v_cache_w : p.k_cache_w);
+      reinterpret_cast<uint4*>(cache + (row * p.S_max + pos) * D)[ch] = val;
+    }
+  }
+  // the stage is refilled by TMA (async proxy) once released: order these writes first
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
 }
 
 template <int D>
@@ -431,8 +465,12 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         if (item < 0 || item >= p.nitems) break;
         const ItemCoord c = item_coord(p, item);
         const int raw = __ldg(p.seqlens + c.b);
-        const int len = valid_len(raw, p.S_max);
-        if (len != raw && c.g == 0 && c.split == 0 && c.hsl == 0) raise_error(GQA_DEVERR_SEQLEN);
+        const int len = valid_len(raw + p.len_add, p.S_max);
+        if (c.g == 0 && c.split == 0 && c.hsl == 0) {
+          if (p.len_add ? (raw < 0 || raw >= p.S_max) : (len != raw)) {
+            raise_error(p.len_add ? GQA_DEVERR_APPEND_POS : GQA_DEVERR_SEQLEN);
+          }
+        }
         const int t_begin = c.split * p.chunk;
         const int t_end = min(len, t_begin + p.chunk);
         if (t_begin >= t_end) {
@@ -450,7 +488,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           if (!ok) break;
           const int t0 = t_begin + tt * kDecTileKeys;
           const int rows = min(kDecTileKeys, t_end - t0);
-          info[s] = StageInfo{item, rows, tt == 0, tt == ntiles - 1};
+          const int new_row = (p.len_add && t0 <= len - 1 && len - 1 < t0 + rows) ? len - 1 - t0 : -1;
+          info[s] = StageInfo{item, rows, (tt == 0 ? 1 : 0) | (tt == ntiles - 1 ? 2 : 0), new_row};
           issue_tile<D>(smem + s * C::kStageBytes, &full[s], &tm_k, &tm_v, row_base + t0, rows, policy);
         }
         if (!ok) break;
@@ -482,15 +521,17 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (!mbar_wait_bounded(&full[s], (it / C::kStages) & 1)) break;  // every consumer warp sees the same barrier
     const StageInfo si = info[s];
     if (si.item < 0) break;
-    if (si.first) {
+    if (si.flags & 1) {
       cur = item_coord(p, si.item);
       load_q_frag<D>(qf, static_cast<const __nv_bfloat16*>(p.q) + ((size_t)cur.b * p.H + cur.h0) * D, lane, cur.nh);
       st.reset();
     }
+    if (si.new_row >= 0 && (si.new_row >> 4) == warp)
+      append_row<D>(p, cur, smem + s * C::kStageBytes, si.new_row, lane);
     if (kb < si.rows) warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-    if (si.last) item_epilogue<D>(p, cur, st, merge, tid, warp, lane);
+    if (si.flags & 2) item_epilogue<D>(p, cur, st, merge, tid, warp, lane);
   }
 }
 
@@ -604,17 +645,18 @@ template <typename OutT, int D>
 __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(OutT* __restrict__ out,
                                                                      const float* __restrict__ ws_o,
                                                                      const float2* __restrict__ ws_ml,
-                                                                     const int32_t* __restrict__ seqlens, int H, int K,
-                                                                     int S_max, int G, int chunk, int nsplit,
-                                                                     int skip_single) {
+                                                                     const int32_t* __restrict__ seqlens, int len_add,
+                                                                     int H, int K, int S_max, int G, int chunk,
+                                                                     int nsplit, int skip_single) {
+  constexpr int kBatch = 8;  // splits per thread group whose rows are loaded up front
   __shared__ float sw[kMaxCombineSplits];
   __shared__ float4 sacc[4][D / 4];
-  __shared__ float sred[2];
+  __shared__ float sred[8];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
   const int g = h / G, j = h % G;
-  const int len = valid_len(__ldg(seqlens + b), S_max);
+  const int len = valid_len(__ldg(seqlens + b) + len_add, S_max);
   const int ns = (len + chunk - 1) / chunk;
   const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
   if (ns == 0) {  // empty sequence
@@ -623,34 +665,54 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(OutT* __re
   }
   if (ns == 1 && skip_single) return;
   const size_t base = ((size_t)(b * K + g) * nsplit) * G + j;  // split s at base + s*G
-  // max and weights
-  float M = -INFINITY;
-  for (int s = tid; s < ns; s += kCombThreads) M = fmaxf(M, __ldcg(&ws_ml[base + (size_t)s * G].x));
+  const bool col = lane < D / 4;
+  // every load of the first round goes out before anything waits on one
+  float2 ml = tid < ns ? __ldcg(&ws_ml[base + (size_t)tid * G]) : make_float2(-INFINITY, 0.f);
+  float4 v[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) {
+    const int s = grp + 4 * u;
+    v[u] = (col && s < ns) ? __ldcg(reinterpret_cast<const float4*>(ws_o + (base + (size_t)s * G) * D) + lane)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // M = max m_s
+  float M = ml.x;
+  for (int s = tid + kCombThreads; s < ns; s += kCombThreads) M = fmaxf(M, __ldcg(&ws_ml[base + (size_t)s * G].x));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  if (lane == 0) sw[grp] = M;
+  if (lane == 0) sred[grp] = M;
   __syncthreads();
-  M = fmaxf(fmaxf(sw[0], sw[1]), fmaxf(sw[2], sw[3]));
-  __syncthreads();
+  M = fmaxf(fmaxf(sred[0], sred[1]), fmaxf(sred[2], sred[3]));
+  // weights 2^(m_s - M) and L = sum l_s 2^(m_s - M)
   float L = 0.f;
-  for (int s = tid; s < ns; s += kCombThreads) {
-    const float2 ml = __ldcg(&ws_ml[base + (size_t)s * G]);
+  if (tid < ns) {
     const float f = fast_exp2(ml.x - M);
+    sw[tid] = f;
+    L = ml.y * f;
+  }
+  for (int s = tid + kCombThreads; s < ns; s += kCombThreads) {
+    const float2 m2 = __ldcg(&ws_ml[base + (size_t)s * G]);
+    const float f = fast_exp2(m2.x - M);
     sw[s] = f;
-    L += ml.y * f;
+    L += m2.y * f;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-  if (lane == 0) sacc[grp][0].x = L;
+  if (lane == 0) sred[4 + grp] = L;
   __syncthreads();
-  if (tid == 0) sred[0] = sacc[0][0].x + sacc[1][0].x + sacc[2][0].x + sacc[3][0].x;
-  __syncthreads();
-  // weighted sum of the partial O rows
+  // weighted sum of the partial O rows: the loaded batch, then any further splits
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (lane < D / 4) {
-    constexpr int kBatch = 8;
-    for (int s0 = grp; s0 < ns; s0 += 4 * kBatch) {
-      float4 v[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) {
+    const int s = grp + 4 * u;
+    const float f = s < ns ? sw[s] : 0.f;
+    acc.x += v[u].x * f;
+    acc.y += v[u].y * f;
+    acc.z += v[u].z * f;
+    acc.w += v[u].w * f;
+  }
+  if (col) {
+    for (int s0 = grp + 4 * kBatch; s0 < ns; s0 += 4 * kBatch) {
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         const int s = s0 + 4 * u;
@@ -671,7 +733,7 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(OutT* __re
   }
   __syncthreads();
   if (tid < D / 4) {
-    const float inv = 1.f / sred[0];
+    const float inv = 1.f / (sred[4] + sred[5] + sred[6] + sred[7]);
     float4 t = sacc[0][tid];
 #pragma unroll
     for (int q = 1; q < 4; ++q) {

@@ -281,15 +281,22 @@ size_t gqa_decode_workspace_bytes(int B, int H, int K, int S_max, int d, int num
   return std::max(a.ws_bytes, b.ws_bytes);
 }
 
-int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
-               int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
-               gqa_dtype dtype, gqa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// gqa_decode, and with append != 0 gqa_decode_append (seqlens then holds pos).
+int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
+                int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                gqa_dtype dtype, gqa_stream_t stream, const void* k_new, const void* v_new, int append) {
   if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
   if (num_splits < 0 || B < 0 || H <= 0 || K <= 0 || S_max <= 0) return GQA_ERR_INVALID_ARG;
   if (!valid_decode_shape(B, H, K, S_max, d)) return GQA_ERR_SHAPE;
   if (B == 0) return GQA_OK;
   if (!out || !q || !k_cache || !v_cache || !seqlens) return GQA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return GQA_ERR_ALIGN;
+  if (append && (!k_new || !v_new)) return GQA_ERR_INVALID_ARG;
+  if (append && (!aligned16(k_new) || !aligned16(v_new))) return GQA_ERR_ALIGN;
   const int dev = current_device();
   const DecodePlan pl = plan_decode(B, H, K, S_max, d, num_splits, dtype, sm_count(dev));
   if (pl.ws_bytes == (size_t)-1) return GQA_ERR_SHAPE;  // more work items than the work counter holds
@@ -299,7 +306,18 @@ int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cach
   }
   const int G = H / K;
   cudaStream_t st = (cudaStream_t)stream;
+  if (append && dtype != GQA_BF16) {  // f32: the append as its own launch, then the decode
+    const int rc = gqa_kv_append(const_cast<void*>(k_cache), const_cast<void*>(v_cache), k_new, v_new, seqlens, B, K,
+                                 S_max, d, dtype, stream);
+    if (rc != GQA_OK) return rc;
+  }
   DecodeParams p;
+  const bool fused_append = append && dtype == GQA_BF16;
+  p.k_new = fused_append ? k_new : nullptr;
+  p.v_new = fused_append ? v_new : nullptr;
+  p.k_cache_w = const_cast<void*>(k_cache);
+  p.v_cache_w = const_cast<void*>(v_cache);
+  p.len_add = append ? 1 : 0;
   p.q = q;
   p.out = out;
   p.ws_o = static_cast<float*>(workspace);
@@ -343,22 +361,40 @@ int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cach
   if (dtype == GQA_BF16)
     e = d == 128 ? cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<__nv_bfloat16, 128>,
                                       static_cast<__nv_bfloat16*>(out), (const float*)p.ws_o, (const float2*)p.ws_ml,
-                                      seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single)
+                                      seqlens, p.len_add, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single)
                  : cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<__nv_bfloat16, 64>,
                                       static_cast<__nv_bfloat16*>(out), (const float*)p.ws_o, (const float2*)p.ws_ml,
-                                      seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single);
+                                      seqlens, p.len_add, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single);
   else
     e = d == 128 ? cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<float, 128>, static_cast<float*>(out),
-                                      (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, H, K, S_max, G, pl.chunk,
+                                      (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, p.len_add, H, K, S_max, G, pl.chunk,
                                       pl.nsplit, skip_single)
                  : cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<float, 64>, static_cast<float*>(out),
-                                      (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, H, K, S_max, G, pl.chunk,
+                                      (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, p.len_add, H, K, S_max, G, pl.chunk,
                                       pl.nsplit, skip_single);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GQA_ERR_CUDA;
   }
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
+               int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+               gqa_dtype dtype, gqa_stream_t stream) {
+  return decode_impl(out, q, k_cache, v_cache, seqlens, B, H, K, S_max, d, scale, num_splits, workspace,
+                     workspace_bytes, dtype, stream, nullptr, nullptr, 0);
+}
+
+int gqa_decode_append(void* out, const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                      const int32_t* pos, int B, int H, int K, int S_max, int d, float scale, int num_splits,
+                      void* workspace, size_t workspace_bytes, gqa_dtype dtype, gqa_stream_t stream) {
+  return decode_impl(out, q, k_cache, v_cache, pos, B, H, K, S_max, d, scale, num_splits, workspace, workspace_bytes,
+                     dtype, stream, k_new, v_new, 1);
 }
 
 int gqa_prefill_causal(void* out, const void* q, const void* k, const void* v, void* k_cache, void* v_cache, int B,

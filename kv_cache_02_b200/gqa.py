@@ -27,8 +27,8 @@ GQA_DEVERR_APPEND_POS, GQA_DEVERR_SEQLEN, GQA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 GQA_ERR_SCRATCH_LIMIT = -7
 GQA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
-EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode", "gqa_decode_noalloc", "gqa_prefill_causal",
-            "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string")
+EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode", "gqa_decode_append", "gqa_decode_noalloc",
+            "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string")
 
 
 class GqaError(RuntimeError):
@@ -49,6 +49,8 @@ def _load():
     lib.gqa_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.gqa_decode.restype = I
     lib.gqa_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, I, P]
+    lib.gqa_decode_append.restype = I
+    lib.gqa_decode_append.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, I, P]
     lib.gqa_decode_noalloc.restype = I
     lib.gqa_decode_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, P]
     lib.gqa_prefill_causal.restype = I
@@ -123,6 +125,21 @@ def gqa_decode(out, q, k_cache, v_cache, seqlens, scale: float, num_splits: int 
     _check("gqa_decode", _lib.gqa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, H, K,
                                          S_max, d, float(scale), int(num_splits), _ptr(workspace), ws_bytes,
                                          _dtype(q), _stream(stream)))
+
+
+def gqa_decode_append(out, q, k_cache, v_cache, k_new, v_new, pos, scale: float, num_splits: int = 0,
+                      workspace=None, stream=None) -> None:
+    """Append k_new/v_new [B,K,d] at row pos[b], then decode over pos[b] + 1 keys (one pass)."""
+    B, H, d = q.shape
+    _, K, S_max, _ = k_cache.shape
+    assert out.shape == q.shape and k_cache.shape[0] == B and k_cache.shape[3] == d
+    assert v_cache.shape == k_cache.shape and k_new.shape == (B, K, d) and v_new.shape == (B, K, d)
+    assert pos.dtype == torch.int32 and pos.shape == (B,)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("gqa_decode_append", _lib.gqa_decode_append(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_new),
+                                                       _ptr(v_new), _ptr(pos), B, H, K, S_max, d, float(scale),
+                                                       int(num_splits), _ptr(workspace), ws_bytes, _dtype(q),
+                                                       _stream(stream)))
 
 
 def gqa_decode_noalloc(out, q, k_cache, v_cache, seqlens, scale: float, num_splits: int = 0, stream=None) -> None:

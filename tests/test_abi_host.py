@@ -28,8 +28,8 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     assert declared_symbols() == sorted(["gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode",
-                                         "gqa_decode_noalloc", "gqa_prefill_causal", "gqa_meanpool_kv",
-                                         "gqa_get_last_error", "gqa_status_string"])
+                                         "gqa_decode_append", "gqa_decode_noalloc", "gqa_prefill_causal",
+                                         "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string"])
 
 
 def test_library_exports_every_declared_symbol(lib):

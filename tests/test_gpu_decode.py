@@ -185,3 +185,73 @@ def test_decode_workspace_needs_no_initialisation(gqa):
             gqa.gqa_decode(out, q, kc, vc, lens, 0.1, 0, ws)
             assert gqa.gqa_get_last_error() == (0, 0)
             assert_close(host(out), ref, f"fill {fill:#x}")
+
+
+# ---------------------------------------------------------------------------
+# gqa_decode_append: the append fused into the decode pass
+
+def run_decode_append(gqa, inp, kn, vn, pos, scale, num_splits=0):
+    q = dev(inp["q"])
+    kc, vc = dev(inp["k_cache"]), dev(inp["v_cache"])
+    B, H, d = inp["q"].shape
+    K, S_max = inp["k_cache"].shape[1], inp["k_cache"].shape[2]
+    ws_bytes = gqa.gqa_decode_workspace_bytes(B, H, K, S_max, d, num_splits)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    out = Guarded((B, H, d), q.dtype)
+    gqa.gqa_decode_append(out.t, q, kc, vc, dev(kn), dev(vn), dev(np.asarray(pos, np.int32)), scale, num_splits, ws)
+    status = gqa.gqa_get_last_error()
+    assert out.intact(), "write outside the output buffer"
+    return host(out.t), host(kc), host(vc), status
+
+
+APPEND = [
+    # B, H, K, d, S_max, pos, dtype
+    (4, 32, 8, 128, 2048, (2047, 1000, 0, 63), synth.BF16),   # token rows at tile edges and at 0
+    (3, 64, 1, 128, 700, (699, 64, 129), synth.BF16),          # MQA: head slices share the row
+    (2, 16, 2, 64, 300, (299, 17), synth.BF16),
+    (2, 8, 2, 64, 128, (127, 5), synth.F32),                   # f32: append launch + decode
+]
+
+
+@pytest.mark.parametrize("num_splits", [0, 1, 5])
+@pytest.mark.parametrize("shape", APPEND, ids=lambda s: f"B{s[0]}H{s[1]}K{s[2]}d{s[3]}S{s[4]}{'f32' if s[6] == synth.F32 else ''}")
+def test_decode_append_equals_append_then_decode(gqa, shape, num_splits):
+    B, H, K, d, S_max, pos, dt = shape
+    pos = np.asarray(pos, np.int32)
+    inp = make(B, H, K, d, S_max, pos, dt, 0xA99E + H + d)  # rows >= pos are NaN before the append
+    kn, vn = synth.normal((B, K, d), dt, 0xA99F, 5), synth.normal((B, K, d), dt, 0xA99F, 6)
+    scale = 1.0 / np.sqrt(d)
+    got, kc, vc, status = run_decode_append(gqa, inp, kn, vn, pos, scale, num_splits)
+    assert status == (0, 0)
+    want_k, want_v = oracle.kv_append(inp["k_cache"], inp["v_cache"], kn, vn, pos)
+    assert np.array_equal(kc.view(np.uint8), want_k.view(np.uint8)) and np.array_equal(vc.view(np.uint8), want_v.view(np.uint8))
+    ref = oracle.decode(inp["q"], want_k, want_v, pos + 1, scale)
+    assert_close(got, ref, f"{shape[:5]} splits={num_splits}")
+
+
+def test_decode_append_bad_position(gqa):
+    B, H, K, d, S_max = 3, 16, 4, 128, 64
+    pos = np.array([S_max, 10, -1], np.int32)
+    inp = make(B, H, K, d, S_max, np.array([S_max, 10, 0], np.int32), synth.BF16, 0xBAD2)
+    kn, vn = synth.normal((B, K, d), synth.BF16, 0xBAD3, 5), synth.normal((B, K, d), synth.BF16, 0xBAD3, 6)
+    got, kc, vc, (status, bits) = run_decode_append(gqa, inp, kn, vn, pos, 0.1)
+    assert status == gqa.GQA_ERR_DEVICE and bits & gqa.GQA_DEVERR_APPEND_POS
+    assert np.all(oracle.widen(got[0]) == 0.0) and np.all(oracle.widen(got[2]) == 0.0)
+    want_k, want_v = oracle.kv_append(inp["k_cache"], inp["v_cache"], kn, vn, pos)
+    assert np.array_equal(kc.view(np.uint8), want_k.view(np.uint8)) and np.array_equal(vc.view(np.uint8), want_v.view(np.uint8))
+    ref = oracle.decode(inp["q"], want_k, want_v, np.array([0, 11, 0], np.int32), 0.1)
+    assert_close(got[1:2], ref[1:2], "valid row next to bad ones")
+
+
+def test_decode_append_full_size_sampled(gqa):
+    w = synth.DECODE_WORKLOADS["llama3_8b_decode_b8_h32_k8_d128_s8192"]
+    inp = synth.decode_inputs(w)
+    scale = 1.0 / np.sqrt(w.d)
+    got, kc, vc, status = run_decode_append(gqa, inp, inp["k_new"], inp["v_new"], inp["pos"], scale)
+    assert status == (0, 0)
+    want_k, want_v = oracle.kv_append(inp["k_cache"], inp["v_cache"], inp["k_new"], inp["v_new"], inp["pos"])
+    assert np.array_equal(kc, want_k) and np.array_equal(vc, want_v)
+    rng = np.random.default_rng(8)
+    sel = np.stack([rng.integers(0, w.B, 48), rng.integers(0, w.H, 48)], 1).astype(np.int32)
+    ref = oracle.decode(inp["q"], want_k, want_v, inp["pos"] + 1, scale, sel=sel)
+    assert_close(got[sel[:, 0], sel[:, 1]], ref, "fused append + decode, Llama-3-8B layer")
