@@ -357,6 +357,19 @@ struct ItemCoord {
   int b, g, unit, split, hsl, h0, nh;
 };
 
+__device__ __forceinline__ ItemCoord item_coord_n(const DecodeParams& p, int item, int heads_per_cta) {
+  ItemCoord c;
+  c.hsl = item % p.hslices;
+  const int rest = item / p.hslices;
+  c.split = rest % p.nsplit;
+  c.unit = rest / p.nsplit;
+  c.b = c.unit / p.K;
+  c.g = c.unit % p.K;
+  c.h0 = c.g * p.G + c.hsl * heads_per_cta;
+  c.nh = min(heads_per_cta, p.G - c.hsl * heads_per_cta);
+  return c;
+}
+
 __device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item) {
   ItemCoord c;
   c.hsl = item % p.hslices;
@@ -460,8 +473,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       int it = 0;  // ring position
       bool ok = true;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-      for (;;) {
-        const int item = take_ticket(p.ws_queue, p.tag) - 1;
+      for (int k = 0;; ++k) {
+        // the first item of each CTA is its block index; later ones come from the counter
+        const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + take_ticket(p.ws_queue, p.tag) - 1;
         if (item < 0 || item >= p.nitems) break;
         const ItemCoord c = item_coord(p, item);
         const int raw = __ldg(p.seqlens + c.b);

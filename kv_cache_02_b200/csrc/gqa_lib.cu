@@ -19,6 +19,7 @@
 #include "append_meanpool.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_wide.cuh"
 #include "prefill.cuh"
 
 namespace {
@@ -86,7 +87,8 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ER
 // decode launch plan
 
 struct DecodePlan {
-  int chunk = 0;       // keys per split (multiple of 64)
+  bool wide = false;   // bf16, d 128, G a multiple of 64: the tcgen05 decode (64 heads per CTA)
+  int chunk = 0;       // keys per split (multiple of the tile)
   int nsplit = 1;      // splits per (b, g)
   int hslices = 1;     // head slices per (b, g)
   long long grid = 0;  // bf16: persistent CTAs; f32: one CTA per work item
@@ -139,25 +141,49 @@ int decode_ctas_per_sm(int dev) {
   return cache[dev];
 }
 
+// Resident wide-group decode CTAs per SM (1 on B200), cached per device.
+int wide_ctas_per_sm(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return 1;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaFuncSetAttribute(gqa::decode_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gqa::WideCfg::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_wide_kernel, gqa::kWideThreads,
+                                                      gqa::WideCfg::kSmemBytes) != cudaSuccess ||
+        n <= 0) {
+      cudaGetLastError();
+      n = 1;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gqa_dtype dt, int sms) {
   DecodePlan pl;
   const int G = H / K;
-  const int heads_per_cta = dt == GQA_BF16 ? gqa::kDecHeadsPerCta : gqa::kDecF32HeadsPerCta;
+  pl.wide = dt == GQA_BF16 && d == 128 && G % gqa::kWideHeads == 0;
+  const int heads_per_cta =
+      pl.wide ? gqa::kWideHeads : (dt == GQA_BF16 ? gqa::kDecHeadsPerCta : gqa::kDecF32HeadsPerCta);
+  const int tile = pl.wide ? gqa::kWideKeys : 64;
   pl.hslices = (G + heads_per_cta - 1) / heads_per_cta;
   const long long units = (long long)B * K * pl.hslices;
-  const int max_splits = std::min((S_max + 63) / 64, gqa::kMaxCombineSplits);
+  const int max_splits = std::min((S_max + tile - 1) / tile, gqa::kMaxCombineSplits);
   int splits;
   if (num_splits > 0) {
     splits = std::min(num_splits, max_splits);
   } else {
-    // about eight work items per SM, never below 256 keys per split
-    const long long target = 8ll * sms;
+    // narrow groups: about eight small work items per SM (their partials are
+    // small); wide groups: about one item per SM, since a 64-head partial is
+    // 32 KB; never below 256 keys per split
+    const long long target = pl.wide ? (long long)sms : 8ll * sms;
     splits = (int)std::max<long long>(1, (target + units - 1) / std::max<long long>(units, 1));
     splits = std::min(splits, std::max(1, (S_max + 255) / 256));
     splits = std::min(splits, max_splits);
   }
   int chunk = (S_max + splits - 1) / splits;
-  chunk = (chunk + 63) / 64 * 64;
+  chunk = (chunk + tile - 1) / tile * tile;
   pl.chunk = chunk;
   pl.nsplit = (S_max + chunk - 1) / chunk;
   const size_t parts = (size_t)B * K * pl.nsplit * G;
@@ -166,7 +192,8 @@ DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gq
   if (dt == GQA_BF16) {
     // persistent CTAs that take work items from a counter in the workspace
     const int dev = current_device();
-    const int per_sm = d == 128 ? decode_ctas_per_sm<128>(dev) : decode_ctas_per_sm<64>(dev);
+    const int per_sm = pl.wide ? wide_ctas_per_sm(dev) : (d == 128 ? decode_ctas_per_sm<128>(dev)
+                                                                    : decode_ctas_per_sm<64>(dev));
     const long long items = units * pl.nsplit;
     pl.grid = std::max<long long>(1, std::min<long long>(items, (long long)per_sm * sms));
     if (items + pl.grid >= (1ll << 24)) {  // beyond the work counter
@@ -192,6 +219,21 @@ int launch_decode_bf16(const DecodePlan& pl, const DecodeParams& p, const void* 
   using C = gqa::DecCfg<D>;
   decode_ctas_per_sm<D>(current_device());  // sets the shared-memory attribute once per device
   gqa::decode_bf16_kernel<D><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(tk, tv, p);
+  return launch_status();
+}
+
+int launch_decode_wide(const DecodePlan& pl, const DecodeParams& p, const void* q, const void* kc, const void* vc,
+                       int B, int H, int K, int S_max, cudaStream_t st) {
+  CUtensorMap tq, tk64, tv64, tk16, tv16;
+  const uint64_t rows = (uint64_t)B * K * S_max;
+  if (!encode_rows_bf16(&tq, q, (uint64_t)B * H, 128, gqa::kWideHeads) ||
+      !encode_rows_bf16(&tk64, kc, rows, 128, gqa::kWideBox) || !encode_rows_bf16(&tv64, vc, rows, 128, gqa::kWideBox) ||
+      !encode_rows_bf16(&tk16, kc, rows, 128, gqa::kDecBoxRows) ||
+      !encode_rows_bf16(&tv16, vc, rows, 128, gqa::kDecBoxRows))
+    return GQA_ERR_CUDA;
+  wide_ctas_per_sm(current_device());  // sets the shared-memory attribute once per device
+  gqa::decode_wide_kernel<<<(unsigned)pl.grid, gqa::kWideThreads, gqa::WideCfg::kSmemBytes, st>>>(tq, tk64, tv64,
+                                                                                                 tk16, tv16, p);
   return launch_status();
 }
 
@@ -306,13 +348,13 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   }
   const int G = H / K;
   cudaStream_t st = (cudaStream_t)stream;
-  if (append && dtype != GQA_BF16) {  // f32: the append as its own launch, then the decode
+  if (append && (dtype != GQA_BF16 || pl.wide)) {  // the append as its own launch, then the decode
     const int rc = gqa_kv_append(const_cast<void*>(k_cache), const_cast<void*>(v_cache), k_new, v_new, seqlens, B, K,
                                  S_max, d, dtype, stream);
     if (rc != GQA_OK) return rc;
   }
   DecodeParams p;
-  const bool fused_append = append && dtype == GQA_BF16;
+  const bool fused_append = append && dtype == GQA_BF16 && !pl.wide;
   p.k_new = fused_append ? k_new : nullptr;
   p.v_new = fused_append ? v_new : nullptr;
   p.k_cache_w = const_cast<void*>(k_cache);
@@ -338,7 +380,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.nsplit = pl.nsplit;
   p.scale_log2 = scale * 1.4426950408889634f;
   int rc;
-  if (dtype == GQA_BF16)
+  if (pl.wide)
+    rc = launch_decode_wide(pl, p, q, k_cache, v_cache, B, H, K, S_max, st);
+  else if (dtype == GQA_BF16)
     rc = d == 128 ? launch_decode_bf16<128>(pl, p, k_cache, v_cache, B, K, S_max, st)
                   : launch_decode_bf16<64>(pl, p, k_cache, v_cache, B, K, S_max, st);
   else

@@ -56,6 +56,8 @@ SMALL = [
     (2, 64, 1, 128, 700, (700, 129)),             # G = 64 (MQA): eight head slices
     (2, 12, 2, 64, 150, (150, 16)),               # G = 6
     (1, 24, 2, 128, 333, (333,)),                 # G = 12: slices of 8 and 4 heads
+    (3, 128, 2, 128, 260, (260, 1, 129)),         # G = 64, two KV heads: the tensor-core wide-group path
+    (2, 128, 1, 128, 500, (500, 300)),            # G = 128: two slices of 64 heads
 ]
 
 
