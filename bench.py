@@ -287,7 +287,12 @@ def bench_ours(args, rank, world, local):
     return result, dict(inp=inp, scale=scale, kv_bytes_layer=kv_bytes_layer)
 
 
-def extra_measurements(args):
+DECODE_EXTRA = ["ragged_70b_decode_b32_h64_k8_d128_s1k_16k", "long_ctx_gqa_b1_h64_k8_d128_s131072",
+                "long_ctx_mqa_b1_h64_k1_d128_s131072"]
+PREFILL = "causal_prefill_b4_s4096_h32_k8_d128"
+
+
+def extra_measurements(args, only=None):
     """Other workloads, rank 0 at N = 1: decode configs and the causal prefill."""
     import torch
 
@@ -295,8 +300,9 @@ def extra_measurements(args):
 
     peaks, _ = measured_peaks()
     res = {}
-    for name in ["ragged_70b_decode_b32_h64_k8_d128_s1k_16k", "long_ctx_gqa_b1_h64_k8_d128_s131072",
-                 "long_ctx_mqa_b1_h64_k1_d128_s131072"]:
+    for name in DECODE_EXTRA:
+        if only is not None and name != only:
+            continue
         w = synth.DECODE_WORKLOADS[name]
         inp = synth.decode_inputs(w)
 
@@ -311,7 +317,7 @@ def extra_measurements(args):
         flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         kv_bytes = int(inp["seqlens"].astype(np.int64).sum()) * w.K * w.d * 2 * 2
         times = []
-        for it in range(args.warmup + 20):
+        for it in range(args.warmup + (args.steps if only else 20)):
             flush.zero_()  # evict the previous iteration's cache rows from L2
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
@@ -326,8 +332,10 @@ def extra_measurements(args):
                      "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "l2": "flushed (512 MiB write)"}
         del q, kc, vc, out, ws, flush
         torch.cuda.empty_cache()
+    if only is not None and only != PREFILL:
+        return res
     # causal prefill with the KV-cache write: FLOPs over the causal pairs (j <= i) only
-    w = synth.PREFILL_WORKLOADS["causal_prefill_b4_s4096_h32_k8_d128"]
+    w = synth.PREFILL_WORKLOADS[PREFILL]
     inp = synth.prefill_inputs(w)
 
     def to_dev2(a):
@@ -339,7 +347,7 @@ def extra_measurements(args):
     vc = torch.empty_like(kc)
     flops = 4.0 * w.B * w.H * w.d * w.S * (w.S + 1) / 2
     times = []
-    for it in range(args.warmup + 20):
+    for it in range(args.warmup + (args.steps if only else 20)):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         gqa.gqa_prefill_causal(out, q, k, v, 1.0 / np.sqrt(w.d), kc, vc)
@@ -412,6 +420,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads and the CPU baseline")
+    ap.add_argument("--only", choices=DECODE_EXTRA + [PREFILL], default=None,
+                    help="time one other workload alone (for profiling); prints its own JSON, not the contract line")
     ap.add_argument("--layers", type=int, default=32,
                     help="layers per step (32 for the model; fewer only for small profiling captures)")
     args = ap.parse_args()
@@ -420,6 +430,10 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_env()
+
+    if args.only:
+        print(json.dumps({"only": args.only, **extra_measurements(args, args.only)}), flush=True)
+        return
 
     if args.impl == "reference":
         res = bench_reference(args, rank, world)

@@ -46,7 +46,7 @@ struct PfCfg {
   static constexpr int kKVOff = kQBytes;
   static constexpr int kPOff = kKVOff + kPfStages * kStageBytes;
   static constexpr int kBarOff = kPOff + kPBytes;
-  static constexpr int kNumBars = 1 + 2 * kPfStages + 2 + 2 + 1 + 1 + 1;
+  static constexpr int kNumBars = 1 + 4 * kPfStages + 2 + 2 + 1 + 1 + 1;
   // at most two CTAs per SM (their 2 x 256 TMEM columns fill the SM's 512)
   static constexpr int kSmemBytes = (kBarOff + kNumBars * 8 + 16) > 80 * 1024 ? (kBarOff + kNumBars * 8 + 16)
                                                                                : 80 * 1024;
@@ -68,9 +68,11 @@ __global__ void __launch_bounds__(kPfThreads, 2)
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* q_full = bars;                  // TMA Q landed
-  uint64_t* kv_full = bars + 1;             // [2] TMA K/V tile landed
-  uint64_t* kv_empty = kv_full + kPfStages; // [2] PV of that tile finished
-  uint64_t* s_full = kv_empty + kPfStages;  // [2] S buffer written by the MMA
+  uint64_t* k_full = bars + 1;              // [2] TMA K tile landed
+  uint64_t* k_empty = k_full + kPfStages;   // [2] S of that tile finished
+  uint64_t* v_full = k_empty + kPfStages;   // [2] TMA V tile landed
+  uint64_t* v_empty = v_full + kPfStages;   // [2] PV of that tile finished
+  uint64_t* s_full = v_empty + kPfStages;   // [2] S buffer written by the MMA
   uint64_t* s_free = s_full + 2;            // [2] S buffer read by all softmax threads
   uint64_t* p_full = s_free + 2;            // P in smem (and O rescaled) for the next PV
   uint64_t* pv_done = p_full + 1;           // the last issued PV finished
@@ -97,8 +99,10 @@ __global__ void __launch_bounds__(kPfThreads, 2)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kPfStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
@@ -120,32 +124,37 @@ __global__ void __launch_bounds__(kPfThreads, 2)
 
   if (warp == 4) {
     // -------------------------------------------------------------- TMA
-    if (lane == 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      const uint64_t pol_q = l2_policy_evict_first();
+    // lane 0 loads Q and the K tiles, lane 1 the V tiles: a K stage is free
+    // again as soon as its S is computed, a V stage only after its PV
+    if (lane < 2) {
+      const bool is_k = lane == 0;
+      const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const int buf_off = C::kKVOff + (is_k ? 0 : C::kTileBytes);
+      prefetch_tensormap(tm);
       const uint64_t pol_kv = l2_policy_evict_last();
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
+      if (is_k) {
+        prefetch_tensormap(&tm_q);
+        const uint64_t pol_q = l2_policy_evict_first();
+        mbar_arrive_expect_tx(q_full, C::kQBytes);
 #pragma unroll
-      for (int hf = 0; hf < C::kHalves; ++hf)
-        tma_load_3d(smem + C::kQOff + hf * C::kQHalf, &tm_q, hf * 64, h, b * p.S + q0, q_full, pol_q);
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_3d(smem + C::kQOff + hf * C::kQHalf, &tm_q, hf * 64, h, b * p.S + q0, q_full, pol_q);
+      }
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kPfStages;
-        if (j >= kPfStages && !mbar_wait_bounded(&kv_empty[s], ((j / kPfStages) - 1) & 1)) break;
-        uint8_t* kd = smem + C::kKVOff + s * C::kStageBytes;
-        uint8_t* vd = kd + C::kTileBytes;
-        mbar_arrive_expect_tx(&kv_full[s], C::kStageBytes);
+        if (j >= kPfStages && !mbar_wait_bounded(&empty[s], ((j / kPfStages) - 1) & 1)) break;
+        uint8_t* dst = smem + buf_off + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], C::kTileBytes);
 #pragma unroll
-        for (int hf = 0; hf < C::kHalves; ++hf) {
-          tma_load_3d(kd + hf * C::kKVHalf, &tm_k, hf * 64, g, b * p.S + j * kPfBN, &kv_full[s], pol_kv);
-          tma_load_3d(vd + hf * C::kKVHalf, &tm_v, hf * 64, g, b * p.S + j * kPfBN, &kv_full[s], pol_kv);
-        }
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_3d(dst + hf * C::kKVHalf, tm, hf * 64, g, b * p.S + j * kPfBN, &full[s], pol_kv);
         ++issued;
       }
       for (int j = max(0, issued - kPfStages); j < issued; ++j)
-        mbar_wait_bounded(&kv_full[j % kPfStages], (j / kPfStages) & 1);
+        mbar_wait_bounded(&full[j % kPfStages], (j / kPfStages) & 1);
     }
   } else if (warp == 5) {
     // -------------------------------------------------------------- MMA
@@ -157,7 +166,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
       bool ok = mbar_wait_bounded(q_full, 0);
       auto issue_s = [&](int j) -> bool {
         const int s = j % kPfStages;
-        if (!mbar_wait_bounded(&kv_full[s], (j / kPfStages) & 1)) return false;
+        if (!mbar_wait_bounded(&k_full[s], (j / kPfStages) & 1)) return false;
         if (j >= 2 && !mbar_wait_bounded(&s_free[j & 1], ((j >> 1) - 1) & 1)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + C::kKVOff + s * C::kStageBytes);
@@ -169,6 +178,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
           tc_mma(tmem + (uint32_t)((j & 1) * kPfBN), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[j & 1]);
+        tc_commit(&k_empty[s]);
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -177,7 +187,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
           ok = false;
           break;
         }
-        if (!mbar_wait_bounded(p_full, j & 1)) {
+        if (!mbar_wait_bounded(p_full, j & 1) || !mbar_wait_bounded(&v_full[j % kPfStages], (j / kPfStages) & 1)) {
           ok = false;
           break;
         }
@@ -190,7 +200,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
           tc_mma(tmem + C::kOCol, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(pv_done);
-        tc_commit(&kv_empty[j % kPfStages]);
+        tc_commit(&v_empty[j % kPfStages]);
       }
       tc_commit(mma_done);
       mbar_wait_bounded(mma_done, 0);
@@ -227,12 +237,24 @@ __global__ void __launch_bounds__(kPfThreads, 2)
 
       const int k0 = j * kPfBN;
       const int kmax = min(qpos, p.S - 1) - k0;  // keys k0 + c with c <= kmax are visible
+      // With a positive scale the maximum is taken on the raw scores and the
+      // scale folds into the exponent (one FFMA per score); off-diagonal
+      // tiles need no mask.
+      const float sl2 = p.scale_log2;
+      const bool pos_scale = sl2 > 0.f;  // the same in every thread
       float mt = -INFINITY;
+      if (pos_scale && kmax >= kPfBN - 1) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        x[c] = c <= kmax ? x[c] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, x[c]);
+        for (int c = 0; c < 64; ++c) mt = fmaxf(mt, x[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          x[c] = c <= kmax ? (pos_scale ? x[c] : x[c] * sl2) : -INFINITY;
+          mt = fmaxf(mt, x[c]);
+        }
       }
+      const float xs = pos_scale ? sl2 : 1.f;  // scale still to apply to x
+      mt *= xs;
       float alpha = 1.f;
       bool rescale = false;
       if (mt > m_used + 8.f) {  // first tile: m_used = -inf
@@ -245,8 +267,8 @@ __global__ void __launch_bounds__(kPfThreads, 2)
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = fast_exp2(x[2 * c] - m_used);
-        const float p1 = fast_exp2(x[2 * c + 1] - m_used);
+        const float p0 = fast_exp2(fmaf(x[2 * c], xs, -m_used));
+        const float p1 = fast_exp2(fmaf(x[2 * c + 1], xs, -m_used));
         sum += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
