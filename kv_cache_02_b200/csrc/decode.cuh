@@ -77,8 +77,8 @@ struct DecodeParams {
   float scale_log2;            // scale * log2(e)
 };
 
-constexpr int kCntBits = 24;
-constexpr int kMaxCombineSplits = 1024;  // splits per unit the combine kernel accepts  // count field of a tagged counter (work items stay below 2^24)
+constexpr int kCntBits = 24;              // count field of a tagged counter (work items stay below 2^24)
+constexpr int kMaxCombineSplits = 1024;  // most splits per unit that a decode plan makes
 
 __device__ __forceinline__ unsigned long long atom_add_relaxed(unsigned long long* p, unsigned long long v) {
   unsigned long long old;
@@ -346,10 +346,14 @@ __device__ __forceinline__ DecItem decode_item(const DecodeParams& p, int heads_
 // the item's first or last. A consumer epilogue (warp merge, output or
 // partial, arrival, combine) overlaps the loads of the next item.
 
+constexpr int kTileFirst = 1;        // the first tile of a work item
+constexpr int kTileLast = 2;         // the last tile of a work item
+constexpr int kUnitSingleSplit = 4;  // the item's unit has one split: its output is final
+
 struct StageInfo {
   int item;     // work item, or -1: no more work
   int rows;     // valid keys in the tile
-  int flags;    // 1: first tile of the item, 2: last tile of the item
+  int flags;    // kTileFirst | kTileLast | kUnitSingleSplit
   int new_row;  // row of the tile that holds the appended token, or -1
 };
 
@@ -387,10 +391,8 @@ __device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item)
 // with a single split) or the split's partial for decode_combine_kernel.
 template <int D>
 __device__ __forceinline__ void item_epilogue(const DecodeParams& p, const ItemCoord& c, const WarpState<D>& st,
-                                              float* merge, int tid, int warp, int lane) {
+                                              float* merge, bool single, int tid, int warp, int lane) {
   __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(p.out) + ((size_t)c.b * p.H + c.h0) * D;
-  const int len = valid_len(__ldg(p.seqlens + c.b) + p.len_add, p.S_max);
-  const int ns = (len + p.chunk - 1) / p.chunk;  // splits that hold keys of this unit
   consumer_bar();  // the previous epilogue has finished with the scratch
   stash_warp_state<D>(merge, st, warp, lane);
   consumer_bar();
@@ -399,7 +401,7 @@ __device__ __forceinline__ void item_epilogue(const DecodeParams& p, const ItemC
     const int h = i / D, dim = i % D;
     float M, L, O;
     merged<D>(merge, h, dim, M, L, O);
-    if (ns == 1) {
+    if (single) {
       out_row[i] = __float2bfloat16_rn(O / L);
     } else {
       p.ws_o[(part + h) * D + dim] = O;
@@ -503,7 +505,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           const int t0 = t_begin + tt * kDecTileKeys;
           const int rows = min(kDecTileKeys, t_end - t0);
           const int new_row = (p.len_add && t0 <= len - 1 && len - 1 < t0 + rows) ? len - 1 - t0 : -1;
-          info[s] = StageInfo{item, rows, (tt == 0 ? 1 : 0) | (tt == ntiles - 1 ? 2 : 0), new_row};
+          info[s] = StageInfo{item, rows,
+                              (tt == 0 ? kTileFirst : 0) | (tt == ntiles - 1 ? kTileLast : 0) |
+                                  (len <= p.chunk ? kUnitSingleSplit : 0),
+                              new_row};
           issue_tile<D>(smem + s * C::kStageBytes, &full[s], &tm_k, &tm_v, row_base + t0, rows, policy);
         }
         if (!ok) break;
@@ -535,7 +540,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (!mbar_wait_bounded(&full[s], (it / C::kStages) & 1)) break;  // every consumer warp sees the same barrier
     const StageInfo si = info[s];
     if (si.item < 0) break;
-    if (si.flags & 1) {
+    if (si.flags & kTileFirst) {
       cur = item_coord(p, si.item);
       load_q_frag<D>(qf, static_cast<const __nv_bfloat16*>(p.q) + ((size_t)cur.b * p.H + cur.h0) * D, lane, cur.nh);
       st.reset();
@@ -545,7 +550,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (kb < si.rows) warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-    if (si.flags & 2) item_epilogue<D>(p, cur, st, merge, tid, warp, lane);
+    if (si.flags & kTileLast) item_epilogue<D>(p, cur, st, merge, (si.flags & kUnitSingleSplit) != 0, tid, warp, lane);
   }
 }
 
@@ -647,56 +652,67 @@ __global__ void __launch_bounds__(kDecF32Threads) decode_f32_kernel(const float*
 // Split-KV combine (the log-sum-exp merge of the partials):
 //   M = max_s m_s,  out[b,h] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s
 // over the ns = ceil(len_b / chunk) splits that hold keys (units with one
-// split were finished by the decode kernel). One CTA of 128 threads per
-// (b, h): four groups of 32 threads take every fourth split, each thread one
-// 16-byte column group, eight loads in flight; the groups are summed in
-// shared memory. Launched as a programmatic dependent of the decode kernel:
-// it waits for that grid before reading the partials.
+// split were finished by the decode kernel). CS CTAs per (b, h), each for
+// D / CS columns; in a CTA of NT threads, RL = D / (4 CS) threads cover one
+// partial row (a 16-byte column group each) and the NT / RL row slots take
+// every (NT / RL)-th split, kBatch rows each loaded before anything waits.
+// Launched as a programmatic dependent of the decode kernel: the length is
+// read before the grid dependency (the decode kernel does not write it), the
+// partials after it.
+template <int D, int NT, int CS>
+struct CombineCfg {
+  static constexpr int RL = D / 4 / CS;  // threads per partial row
+  static constexpr int R = NT / RL;      // row slots
+  static constexpr int kBatch = (160 + R - 1) / R < 8 ? (160 + R - 1) / R : 8;  // up to 160 rows in the first round
+  static_assert(RL >= 1 && RL <= 32 && NT % RL == 0 && NT % 32 == 0, "combine shape");
+};
 
-constexpr int kCombThreads = 128;
-
-template <typename OutT, int D>
-__global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(OutT* __restrict__ out,
-                                                                     const float* __restrict__ ws_o,
-                                                                     const float2* __restrict__ ws_ml,
-                                                                     const int32_t* __restrict__ seqlens, int len_add,
-                                                                     int H, int K, int S_max, int G, int chunk,
-                                                                     int nsplit, int skip_single) {
-  constexpr int kBatch = 8;  // splits per thread group whose rows are loaded up front
+template <typename OutT, int D, int NT, int CS>
+__global__ void __launch_bounds__(NT) decode_combine_kernel(OutT* __restrict__ out, const float* __restrict__ ws_o,
+                                                            const float2* __restrict__ ws_ml,
+                                                            const int32_t* __restrict__ seqlens, int len_add, int H,
+                                                            int K, int S_max, int G, int chunk, int nsplit,
+                                                            int skip_single) {
+  using CC = CombineCfg<D, NT, CS>;
+  constexpr int RL = CC::RL, R = CC::R, kBatch = CC::kBatch, NW = NT / 32;
   __shared__ float sw[kMaxCombineSplits];
-  __shared__ float4 sacc[4][D / 4];
-  __shared__ float sred[8];
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int bh = blockIdx.x;
+  __shared__ float4 sacc[R][RL];
+  __shared__ float sred[2 * NW];
+  const int bh = blockIdx.x / CS, slice = blockIdx.x % CS;
   const int b = bh / H, h = bh % H;
   const int g = h / G, j = h % G;
   const int len = valid_len(__ldg(seqlens + b) + len_add, S_max);
   const int ns = (len + chunk - 1) / chunk;
-  const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int col = tid % RL, slot = tid / RL;
+  OutT* orow = out + (size_t)bh * D + slice * (D / CS);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (ns == 0) {  // empty sequence
-    for (int i = tid; i < D; i += kCombThreads) store_out<OutT>(out + (size_t)bh * D + i, 0.f);
+    for (int i = tid; i < D / CS; i += NT) store_out<OutT>(orow + i, 0.f);
     return;
   }
   if (ns == 1 && skip_single) return;
   const size_t base = ((size_t)(b * K + g) * nsplit) * G + j;  // split s at base + s*G
-  const bool col = lane < D / 4;
+  const float* obase = ws_o + base * D + slice * (D / CS);
   // every load of the first round goes out before anything waits on one
   float2 ml = tid < ns ? __ldcg(&ws_ml[base + (size_t)tid * G]) : make_float2(-INFINITY, 0.f);
   float4 v[kBatch];
 #pragma unroll
   for (int u = 0; u < kBatch; ++u) {
-    const int s = grp + 4 * u;
-    v[u] = (col && s < ns) ? __ldcg(reinterpret_cast<const float4*>(ws_o + (base + (size_t)s * G) * D) + lane)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int sp = slot + R * u;
+    v[u] = sp < ns ? __ldcg(reinterpret_cast<const float4*>(obase + (size_t)sp * G * D) + col)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   // M = max m_s
   float M = ml.x;
-  for (int s = tid + kCombThreads; s < ns; s += kCombThreads) M = fmaxf(M, __ldcg(&ws_ml[base + (size_t)s * G].x));
+  for (int sp = tid + NT; sp < ns; sp += NT) M = fmaxf(M, __ldcg(&ws_ml[base + (size_t)sp * G].x));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  if (lane == 0) sred[grp] = M;
+  if (lane == 0) sred[warp] = M;
   __syncthreads();
-  M = fmaxf(fmaxf(sred[0], sred[1]), fmaxf(sred[2], sred[3]));
+  M = sred[0];
+#pragma unroll
+  for (int q = 1; q < NW; ++q) M = fmaxf(M, sred[q]);
   // weights 2^(m_s - M) and L = sum l_s 2^(m_s - M)
   float L = 0.f;
   if (tid < ns) {
@@ -704,59 +720,60 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(OutT* __re
     sw[tid] = f;
     L = ml.y * f;
   }
-  for (int s = tid + kCombThreads; s < ns; s += kCombThreads) {
-    const float2 m2 = __ldcg(&ws_ml[base + (size_t)s * G]);
+  for (int sp = tid + NT; sp < ns; sp += NT) {
+    const float2 m2 = __ldcg(&ws_ml[base + (size_t)sp * G]);
     const float f = fast_exp2(m2.x - M);
-    sw[s] = f;
+    sw[sp] = f;
     L += m2.y * f;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-  if (lane == 0) sred[4 + grp] = L;
+  if (lane == 0) sred[NW + warp] = L;
   __syncthreads();
   // weighted sum of the partial O rows: the loaded batch, then any further splits
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int u = 0; u < kBatch; ++u) {
-    const int s = grp + 4 * u;
-    const float f = s < ns ? sw[s] : 0.f;
+    const int sp = slot + R * u;
+    const float f = sp < ns ? sw[sp] : 0.f;
     acc.x += v[u].x * f;
     acc.y += v[u].y * f;
     acc.z += v[u].z * f;
     acc.w += v[u].w * f;
   }
-  if (col) {
-    for (int s0 = grp + 4 * kBatch; s0 < ns; s0 += 4 * kBatch) {
+  for (int s0 = slot + R * kBatch; s0 < ns; s0 += R * kBatch) {
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int s = s0 + 4 * u;
-        v[u] = s < ns ? __ldcg(reinterpret_cast<const float4*>(ws_o + (base + (size_t)s * G) * D) + lane)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int s = s0 + 4 * u;
-        const float f = s < ns ? sw[s] : 0.f;
-        acc.x += v[u].x * f;
-        acc.y += v[u].y * f;
-        acc.z += v[u].z * f;
-        acc.w += v[u].w * f;
-      }
+    for (int u = 0; u < kBatch; ++u) {
+      const int sp = s0 + R * u;
+      v[u] = sp < ns ? __ldcg(reinterpret_cast<const float4*>(obase + (size_t)sp * G * D) + col)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    sacc[grp][lane] = acc;
-  }
-  __syncthreads();
-  if (tid < D / 4) {
-    const float inv = 1.f / (sred[4] + sred[5] + sred[6] + sred[7]);
-    float4 t = sacc[0][tid];
 #pragma unroll
-    for (int q = 1; q < 4; ++q) {
+    for (int u = 0; u < kBatch; ++u) {
+      const int sp = s0 + R * u;
+      const float f = sp < ns ? sw[sp] : 0.f;
+      acc.x += v[u].x * f;
+      acc.y += v[u].y * f;
+      acc.z += v[u].z * f;
+      acc.w += v[u].w * f;
+    }
+  }
+  sacc[slot][col] = acc;
+  __syncthreads();
+  if (tid < RL) {
+    float Lt = 0.f;
+#pragma unroll
+    for (int q = 0; q < NW; ++q) Lt += sred[NW + q];
+    const float inv = 1.f / Lt;
+    float4 t = sacc[0][tid];
+#pragma unroll 8
+    for (int q = 1; q < R; ++q) {
       t.x += sacc[q][tid].x;
       t.y += sacc[q][tid].y;
       t.z += sacc[q][tid].z;
       t.w += sacc[q][tid].w;
     }
-    OutT* o = out + (size_t)bh * D + tid * 4;
+    OutT* o = orow + tid * 4;
     store_out<OutT>(o + 0, t.x * inv);
     store_out<OutT>(o + 1, t.y * inv);
     store_out<OutT>(o + 2, t.z * inv);

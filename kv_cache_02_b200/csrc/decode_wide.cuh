@@ -6,8 +6,9 @@
 // 64 heads of a group from every K/V tile it loads:
 //   S[64 heads x 128 keys] = Q[64 x d] K^T[d x 128]    tcgen05.mma M=64, fp32 in TMEM
 //   softmax over keys: an M=64 accumulator puts row r in TMEM lane
-//       (r mod 16) + 32 * (r / 16), so lanes 0..15 of the four softmax warps
-//       each own one head's whole row: max, exp2 and sum stay in the thread
+//       (r mod 16) + 32 * (r / 16); the 16-lane TMEM load shape spreads the
+//       16 rows of a softmax warp over all its 32 threads, a quad of threads
+//       per pair of heads, each thread 32 keys of both
 //   P (bf16) into shared memory as the K-major operand
 //   O[64 x d] += P[64 x 128 keys] V[128 keys x d]      tcgen05.mma, V MN-major
 // The accumulator is rescaled (conditionally, when a head's maximum grows by
@@ -77,6 +78,84 @@ __device__ __forceinline__ void wide_issue_tile(uint8_t* stage, uint64_t* full, 
     }
 }
 
+// One tile of the online softmax for the two heads a thread holds. x: the raw
+// scores of 32 keys of head a (x[4i], x[4i+1]) and of head b (x[4i+2],
+// x[4i+3]), key 8i + 2 qi + {0, 1}. Keys at or past `rows` do not count. The
+// running maxima m_a, m_b are in log2 units with the scale applied and are
+// common to the quad; l_a, l_b are this thread's share of the sums. alpha_a,
+// alpha_b: the factors O must be multiplied by (1 when the maximum is kept).
+// With a positive scale the maximum is taken over the raw scores and the
+// scale folds into the exponent's multiply-add.
+template <bool kPosScale>
+__device__ __forceinline__ void wide_softmax_tile(float (&x)[64], int rows, int qi, float sl2, float& m_a,
+                                                  float& m_b, float& l_a, float& l_b, uint32_t (&pa)[16],
+                                                  uint32_t (&pb)[16], float& alpha_a, float& alpha_b) {
+  if constexpr (!kPosScale) {
+#pragma unroll
+    for (int e = 0; e < 64; ++e) x[e] *= sl2;
+  }
+  if (rows < kWideKeys) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (8 * i + 2 * qi + (k & 1) >= rows) x[4 * i + k] = -INFINITY;
+  }
+  float a0 = x[0], a1 = x[1], b0 = x[2], b1 = x[3];
+#pragma unroll
+  for (int i = 1; i < 16; ++i) {
+    a0 = fmaxf(a0, x[4 * i]);
+    a1 = fmaxf(a1, x[4 * i + 1]);
+    b0 = fmaxf(b0, x[4 * i + 2]);
+    b1 = fmaxf(b1, x[4 * i + 3]);
+  }
+  float ma = fmaxf(a0, a1), mb = fmaxf(b0, b1);
+#pragma unroll
+  for (int off = 1; off <= 2; off <<= 1) {
+    ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, off));
+    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
+  }
+  if constexpr (kPosScale) {
+    ma *= sl2;
+    mb *= sl2;
+  }
+  alpha_a = 1.f;
+  alpha_b = 1.f;
+  if (ma > m_a + 8.f) {  // first tile of an item: m = -inf
+    const float mn = fmaxf(ma, m_a);
+    alpha_a = fast_exp2(m_a - mn);
+    m_a = mn;
+  }
+  if (mb > m_b + 8.f) {
+    const float mn = fmaxf(mb, m_b);
+    alpha_b = fast_exp2(m_b - mn);
+    m_b = mn;
+  }
+  const float nma = -m_a, nmb = -m_b;
+  float sa = 0.f, sb = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float p0, p1, p2, p3;
+    if constexpr (kPosScale) {
+      p0 = fast_exp2(fmaf(x[4 * i], sl2, nma));
+      p1 = fast_exp2(fmaf(x[4 * i + 1], sl2, nma));
+      p2 = fast_exp2(fmaf(x[4 * i + 2], sl2, nmb));
+      p3 = fast_exp2(fmaf(x[4 * i + 3], sl2, nmb));
+    } else {
+      p0 = fast_exp2(x[4 * i] + nma);
+      p1 = fast_exp2(x[4 * i + 1] + nma);
+      p2 = fast_exp2(x[4 * i + 2] + nmb);
+      p3 = fast_exp2(x[4 * i + 3] + nmb);
+    }
+    sa += p0 + p1;
+    sb += p2 + p3;
+    pa[i] = pack_bf16x2(p0, p1);
+    pb[i] = pack_bf16x2(p2, p3);
+  }
+  l_a = l_a * alpha_a + sa;
+  l_b = l_b * alpha_b + sb;
+}
+
 __global__ void __launch_bounds__(kWideThreads, 1)
     decode_wide_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k64,
                        const __grid_constant__ CUtensorMap tm_v64, const __grid_constant__ CUtensorMap tm_k16,
@@ -102,6 +181,15 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) raise_error(GQA_DEVERR_TIMEOUT);
     return;
+  }
+  // the producer fetches its first item's length before the set-up below,
+  // which hides the load's latency
+  int raw_first = 0;
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k64);
+    prefetch_tensormap(&tm_v64);
+    if ((int)blockIdx.x < p.nitems) raw_first = __ldg(p.seqlens + item_coord_n(p, blockIdx.x, kWideHeads).b);
   }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -133,9 +221,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k64);
-      prefetch_tensormap(&tm_v64);
       const uint64_t policy = l2_policy_evict_first();
       const uint64_t q_policy = l2_policy_evict_last();
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
@@ -146,7 +231,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + take_ticket(p.ws_queue, p.tag) - 1;
         if (item < 0 || item >= p.nitems) break;
         const ItemCoord c = item_coord_n(p, item, kWideHeads);
-        const int raw = __ldg(p.seqlens + c.b);
+        const int raw = k == 0 ? raw_first : __ldg(p.seqlens + c.b);
         const int len = valid_len(raw + p.len_add, p.S_max);
         if (c.g == 0 && c.split == 0 && c.hsl == 0 && !p.len_add && len != raw) raise_error(GQA_DEVERR_SEQLEN);
         const int t_begin = c.split * p.chunk;
@@ -173,7 +258,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           if (!ok) break;
           const int t0 = t_begin + tt * kWideKeys;
           const int rows = min(kWideKeys, t_end - t0);
-          info[s] = StageInfo{item, rows, (tt == 0 ? 1 : 0) | (tt == ntiles - 1 ? 2 : 0), -1};
+          info[s] = StageInfo{item, rows,
+                              (tt == 0 ? kTileFirst : 0) | (tt == ntiles - 1 ? kTileLast : 0) |
+                                  (len <= p.chunk ? kUnitSingleSplit : 0),
+                              -1};
           wide_issue_tile(smem + C::kKVOff + s * C::kStage, &kv_full[s], &tm_k64, &tm_v64, &tm_k16, &tm_v16,
                           row_base + t0, rows, policy);
         }
@@ -223,7 +311,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         if (!(ok = mbar_wait_bounded(&kv_full[s], (j / C::kStages) & 1))) break;
         const StageInfo si = info[s];
         if (si.item < 0) break;
-        if (si.flags & 1) {
+        if (si.flags & kTileFirst) {
           if (!(ok = mbar_wait_bounded(q_full, nitem & 1))) break;
           cur_ord = nitem++;
         }
@@ -238,9 +326,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           tc_mma(tmem + C::kSCol + (uint32_t)((j & 1) * kWideKeys), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[j & 1]);
-        if (si.flags & 2) tc_commit(q_empty);  // the item's last S: Q may be replaced
+        if (si.flags & kTileLast) tc_commit(q_empty);  // the item's last S: Q may be replaced
         if (j >= 1 && !(ok = issue_pv(j - 1, prev_first, prev_ord))) break;
-        prev_first = si.flags & 1;
+        prev_first = si.flags & kTileFirst;
         prev_ord = cur_ord;
       }
       if (ok && j >= 1) issue_pv(j - 1, prev_first, prev_ord);
@@ -249,82 +337,64 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     }
   } else {
     // ---------------------------------------------------- softmax / epilogue
-    // lanes 0..15 of warp w own head r = 16 w + lane (TMEM lane 32 w + lane);
-    // lanes 16..31 run the same instructions on rows that hold no head
+    // warp w serves heads 16 w .. 16 w + 15 (TMEM lanes 32 w .. 32 w + 15):
+    // the quad of lanes 4 g .. 4 g + 3 holds heads ra = 16 w + g and
+    // rb = ra + 8, each thread keys 8 i + 2 (lane % 4) + {0, 1} of a tile
     const int t = threadIdx.x;
-    const int r = warp * 16 + (lane & 15);
-    const bool owner = lane < 16;
+    const int g = lane >> 2, qi = lane & 3;
+    const int ra = warp * 16 + g, rb = ra + 8;
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    uint8_t* prow = smem + C::kPOff + r * 128;
-    float m_used = -INFINITY, l = 0.f;
+    uint8_t* prow_a = smem + C::kPOff + ra * 128;
+    uint8_t* prow_b = smem + C::kPOff + rb * 128;
+    const float sl2 = p.scale_log2;
+    const bool pos_scale = sl2 > 0.f;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
     ItemCoord c{};
     for (int j = 0;; ++j) {
       const int s = j % C::kStages;
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&kv_full[s], (j / C::kStages) & 1))) break;
       const StageInfo si = info[s];
       if (si.item < 0) break;
-      const bool first = si.flags & 1;
+      const bool first = si.flags & kTileFirst;
       if (first) {
         c = item_coord_n(p, si.item, kWideHeads);
-        m_used = -INFINITY;
-        l = 0.f;
+        m_a = m_b = -INFINITY;
+        l_a = l_b = 0.f;
       }
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[j & 1], (j >> 1) & 1))) break;
       tc_fence_after();
-      float x[2 * 64];
-      {
-        float a[64], bb[64];
-        tmem_ld64(lane_addr + C::kSCol + (uint32_t)((j & 1) * kWideKeys), a);
-        tmem_ld64(lane_addr + C::kSCol + (uint32_t)((j & 1) * kWideKeys + 64), bb);
-        tc_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          x[i] = a[i];
-          x[64 + i] = bb[i];
-        }
-      }
+      float x[64];
+      tmem_ld_16x256b_x16(lane_addr + C::kSCol + (uint32_t)((j & 1) * kWideKeys), x);
+      tc_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_free[j & 1]);
 
-      float mt = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < kWideKeys; ++k) {
-        x[k] = k < si.rows ? x[k] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, x[k]);
-      }
-      float alpha = 1.f;
-      bool rescale = false;
-      if (mt > m_used + 8.f) {  // first tile of an item: m_used = -inf
-        const float mn = fmaxf(mt, m_used);
-        alpha = fast_exp2(m_used - mn);
-        rescale = !first;
-        m_used = mn;
-      }
-      float sum = 0.f;
-      uint32_t pk[kWideKeys / 2];
-#pragma unroll
-      for (int k = 0; k < kWideKeys; k += 2) {
-        const float p0 = fast_exp2(x[k] - m_used);
-        const float p1 = fast_exp2(x[k + 1] - m_used);
-        sum += p0 + p1;
-        pk[k / 2] = pack_bf16x2(p0, p1);
-      }
-      l = l * alpha + sum;
+      uint32_t pa[16], pb[16];
+      float alpha_a, alpha_b;
+      if (pos_scale)
+        wide_softmax_tile<true>(x, si.rows, qi, sl2, m_a, m_b, l_a, l_b, pa, pb, alpha_a, alpha_b);
+      else
+        wide_softmax_tile<false>(x, si.rows, qi, sl2, m_a, m_b, l_a, l_b, pa, pb, alpha_a, alpha_b);
       // the P buffer and O are free once the previous tile's PV has finished
       if (j >= 1) {
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, (j - 1) & 1))) break;
         tc_fence_after();
       }
-      if (__any_sync(0xffffffffu, rescale && owner)) {  // lanes that keep their max scale by 1
-        const float a = (rescale && owner) ? alpha : 1.f;
+      // a head whose maximum moved (never on an item's first tile, where PV overwrites O)
+      if (__any_sync(0xffffffffu, !first && (alpha_a != 1.f || alpha_b != 1.f))) {
         float o[32];
 #pragma unroll 1
-        for (int cb = 0; cb < D; cb += 32) {
-          tmem_ld32(lane_addr + C::kOCol + cb, o);
+        for (int cb = 0; cb < D; cb += 64) {
+          tmem_ld_16x256b_x8(lane_addr + C::kOCol + cb, o);
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= a;
-          tmem_st32(lane_addr + C::kOCol + cb, o);
+          for (int i = 0; i < 8; ++i) {
+            o[4 * i] *= alpha_a;
+            o[4 * i + 1] *= alpha_a;
+            o[4 * i + 2] *= alpha_b;
+            o[4 * i + 3] *= alpha_b;
+          }
+          tmem_st_16x256b_x8(lane_addr + C::kOCol + cb, o);
         }
         tc_wait_st();
       }
@@ -336,46 +406,54 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           for (int ch = 0; ch < 8; ++ch)
             *reinterpret_cast<uint4*>(vrow + hf * C::kHalf + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
       }
-      if (owner) {
+      // P rows, K-major with the 128-byte swizzle: keys 8 i .. 8 i + 7 form 16-byte chunk i
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          const uint32_t off = (uint32_t)((ch >> 3) * C::kPHalf) + ((((uint32_t)(ch & 7)) ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(prow + off) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        }
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t off = (uint32_t)((i >> 3) * C::kPHalf) + ((((uint32_t)(i & 7)) ^ (uint32_t)g) << 4) + 4u * qi;
+        *reinterpret_cast<uint32_t*>(prow_a + off) = pa[i];
+        *reinterpret_cast<uint32_t*>(prow_b + off) = pb[i];
       }
       fence_async_shared();
       tc_fence_before();
       mbar_arrive(p_full);
 
-      if (si.flags & 2) {
+      if (si.flags & kTileLast) {
         // ---- item epilogue: O / l -> out (one split) or the split's partial
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, j & 1))) break;
         tc_fence_after();
-        float o[D];
-        tmem_ld64(lane_addr + C::kOCol, *reinterpret_cast<float(*)[64]>(o));
-        tmem_ld64(lane_addr + C::kOCol + 64, *reinterpret_cast<float(*)[64]>(o + 64));
+        float o[64];
+        tmem_ld_16x256b_x16(lane_addr + C::kOCol, o);
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(o_free);
-        const int len = valid_len(__ldg(p.seqlens + c.b) + p.len_add, p.S_max);
-        const int ns = (len + p.chunk - 1) / p.chunk;
-        if (owner && ns == 1) {
-          const float inv = 1.f / l;
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                ((size_t)c.b * p.H + c.h0 + r) * D);
+        float la = l_a, lb = l_b;
 #pragma unroll
-          for (int i = 0; i < D / 8; ++i)
-            dst[i] = make_uint4(pack_bf16x2(o[8 * i] * inv, o[8 * i + 1] * inv),
-                                pack_bf16x2(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
-                                pack_bf16x2(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
-                                pack_bf16x2(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
-        } else if (owner) {
-          const size_t part = ((size_t)c.unit * p.nsplit + c.split) * p.G + (size_t)c.hsl * kWideHeads + r;
-          float4* dst = reinterpret_cast<float4*>(p.ws_o + part * D);
+        for (int off = 1; off <= 2; off <<= 1) {
+          la += __shfl_xor_sync(0xffffffffu, la, off);
+          lb += __shfl_xor_sync(0xffffffffu, lb, off);
+        }
+        if (si.flags & kUnitSingleSplit) {
+          const float ia = 1.f / la, ib = 1.f / lb;
+          __nv_bfloat16* oa = static_cast<__nv_bfloat16*>(p.out) + ((size_t)c.b * p.H + c.h0 + ra) * D + 2 * qi;
+          __nv_bfloat16* ob = oa + 8 * D;
 #pragma unroll
-          for (int i = 0; i < D / 4; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-          p.ws_ml[part] = make_float2(m_used, l);
+          for (int i = 0; i < 16; ++i) {
+            *reinterpret_cast<uint32_t*>(oa + 8 * i) = pack_bf16x2(o[4 * i] * ia, o[4 * i + 1] * ia);
+            *reinterpret_cast<uint32_t*>(ob + 8 * i) = pack_bf16x2(o[4 * i + 2] * ib, o[4 * i + 3] * ib);
+          }
+        } else {
+          const size_t part = ((size_t)c.unit * p.nsplit + c.split) * p.G + (size_t)c.hsl * kWideHeads + ra;
+          float* da = p.ws_o + part * D + 2 * qi;
+          float* db = da + 8 * D;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            *reinterpret_cast<float2*>(da + 8 * i) = make_float2(o[4 * i], o[4 * i + 1]);
+            *reinterpret_cast<float2*>(db + 8 * i) = make_float2(o[4 * i + 2], o[4 * i + 3]);
+          }
+          if (qi == 0) {
+            p.ws_ml[part] = make_float2(m_a, la);
+            p.ws_ml[part + 8] = make_float2(m_b, lb);
+          }
         }
       }
     }

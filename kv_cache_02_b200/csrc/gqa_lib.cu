@@ -327,6 +327,49 @@ size_t gqa_decode_workspace_bytes(int B, int H, int K, int S_max, int d, int num
 
 namespace {
 
+template <typename OutT, int D, int NT, int CS>
+cudaError_t launch_combine_t(void* out, const DecodeParams& p, const int32_t* seqlens, int H, int K, int S_max, int G,
+                             int chunk, int nsplit, int skip_single, long long units, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(units * CS));
+  cfg.blockDim = dim3(NT);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<OutT, D, NT, CS>, static_cast<OutT*>(out),
+                            (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, p.len_add, H, K, S_max, G, chunk,
+                            nsplit, skip_single);
+}
+
+// Few splits: one CTA of 128 threads per (b, h). Many splits: four CTAs of
+// 256 threads per (b, h), a quarter of the columns each, so that more SMs
+// share the partial rows and all of them are loaded in one round.
+template <typename OutT, int D>
+cudaError_t launch_combine_d(void* out, const DecodeParams& p, const int32_t* seqlens, int H, int K, int S_max, int G,
+                             int chunk, int nsplit, int skip_single, bool many, long long units, cudaStream_t st) {
+  return many ? launch_combine_t<OutT, D, 256, 4>(out, p, seqlens, H, K, S_max, G, chunk, nsplit, skip_single, units,
+                                                  st)
+              : launch_combine_t<OutT, D, 128, 1>(out, p, seqlens, H, K, S_max, G, chunk, nsplit, skip_single, units,
+                                                  st);
+}
+
+cudaError_t launch_combine(void* out, const DecodeParams& p, const int32_t* seqlens, int H, int K, int S_max, int G,
+                           int chunk, int nsplit, int skip_single, int d, gqa_dtype dt, bool many, long long units,
+                           cudaStream_t st) {
+  if (dt == GQA_BF16)
+    return d == 128 ? launch_combine_d<__nv_bfloat16, 128>(out, p, seqlens, H, K, S_max, G, chunk, nsplit, skip_single,
+                                                           many, units, st)
+                    : launch_combine_d<__nv_bfloat16, 64>(out, p, seqlens, H, K, S_max, G, chunk, nsplit, skip_single,
+                                                          many, units, st);
+  return d == 128 ? launch_combine_d<float, 128>(out, p, seqlens, H, K, S_max, G, chunk, nsplit, skip_single, many,
+                                                 units, st)
+                  : launch_combine_d<float, 64>(out, p, seqlens, H, K, S_max, G, chunk, nsplit, skip_single, many,
+                                                units, st);
+}
+
 // gqa_decode, and with append != 0 gqa_decode_append (seqlens then holds pos).
 int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
                 int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
@@ -391,31 +434,10 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   if (rc != GQA_OK || pl.nsplit == 1) return rc;
   // the split-KV combine, as a programmatic dependent launch: its launch
   // overlaps the decode kernel, and it waits for that grid before reading
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((long long)B * H));
-  cfg.blockDim = dim3(gqa::kCombThreads);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e;
   const int skip_single = dtype == GQA_BF16 ? 1 : 0;  // bf16 units with one split are already written
-  if (dtype == GQA_BF16)
-    e = d == 128 ? cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<__nv_bfloat16, 128>,
-                                      static_cast<__nv_bfloat16*>(out), (const float*)p.ws_o, (const float2*)p.ws_ml,
-                                      seqlens, p.len_add, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single)
-                 : cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<__nv_bfloat16, 64>,
-                                      static_cast<__nv_bfloat16*>(out), (const float*)p.ws_o, (const float2*)p.ws_ml,
-                                      seqlens, p.len_add, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single);
-  else
-    e = d == 128 ? cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<float, 128>, static_cast<float*>(out),
-                                      (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, p.len_add, H, K, S_max, G, pl.chunk,
-                                      pl.nsplit, skip_single)
-                 : cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<float, 64>, static_cast<float*>(out),
-                                      (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, p.len_add, H, K, S_max, G, pl.chunk,
-                                      pl.nsplit, skip_single);
+  const bool many = pl.nsplit > 32;
+  cudaError_t e = launch_combine(out, p, seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single, d, dtype, many,
+                                 (long long)B * H, st);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GQA_ERR_CUDA;
