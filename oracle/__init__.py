@@ -18,6 +18,18 @@ Page citations (title, section):
   * KV append: "分組查詢注意力", section 技術原理 (each new token writes K and
     V of shape [batch, 1, K, d_k]); "GQA 完全拆解", section 解码推理的内存账本
     (after step t the new K, V row is appended to the cache).
+  * Paged KV cache: "分組查詢注意力", section 下游 / 推論引擎與架構 (the
+    paged cache manages blocks of the K KV heads, not of the H query heads,
+    and each block is broadcast to the group's H/K query heads when it is
+    used); "GQA 完全拆解", section 工程实现：权重布局、repeat 与 Kernel 融合 (the
+    block layout is organised by KV head) and section 主流模型里的 GQA：KV 缓存账本
+    (paging removes allocation fragmentation and is orthogonal to GQA); "GQA"
+    (kongchang.com), list of facts (the KV cache is managed in blocks). The
+    pages give no block size or table format; the reading used here is a pool
+    [num_blocks, K, block_size, d] and a table [B, max_blocks] of physical
+    block numbers, logical block i of sequence b holding its keys
+    i * block_size .. (i + 1) * block_size - 1. A paged decode is, by that
+    definition, the decode of the cache the table gathers.
 
 Parity status: pinned (tests/test_oracle_pins.py); nothing here is "parity
 unpinned".
@@ -234,3 +246,55 @@ def prefill_cache_write(k, v, S_max: int, k_cache=None, v_cache=None):
     kc[:, :, :S, :] = np.transpose(k, (0, 2, 1, 3))
     vc[:, :, :S, :] = np.transpose(v, (0, 2, 1, 3))
     return kc, vc
+
+
+# ---------------------------------------------------------------------------
+# paged KV cache: a block table over a pool of blocks (index arithmetic only)
+
+def paged_gather(pool, block_table) -> np.ndarray:
+    """pool [num_blocks, K, bs, d], block_table [B, max_blocks] -> cache [B, K, max_blocks * bs, d].
+
+    cache[b, g, i * bs + r] = pool[block_table[b, i], g, r]. A table entry
+    outside [0, num_blocks) gives NaN rows (no key of a valid length may
+    point there).
+    """
+    pool = _c(pool)
+    table = np.ascontiguousarray(block_table, dtype=np.int64)
+    nb, K, bs, d = pool.shape
+    B, mb = table.shape
+    out = np.empty((B, K, mb * bs, d), dtype=pool.dtype)
+    nan = np.uint16(0x7FC0) if pool.dtype == np.uint16 else np.nan  # a quiet NaN (bfloat16 bits or float)
+    for b in range(B):
+        for i in range(mb):
+            blk = int(table[b, i])
+            if 0 <= blk < nb:
+                out[b, :, i * bs:(i + 1) * bs, :] = pool[blk]
+            else:
+                out[b, :, i * bs:(i + 1) * bs, :] = nan
+    return out
+
+
+def decode_paged(q, k_pool, v_pool, block_table, seqlens, scale: float, sel=None, nthreads=None,
+                 lib=None) -> np.ndarray:
+    """q [B,H,d], pools [num_blocks,K,bs,d], block_table [B,max_blocks], seqlens [B] -> float64 [B,H,d]
+    (or [len(sel), d]): the decode of the cache that the table gathers."""
+    return decode(q, paged_gather(k_pool, block_table), paged_gather(v_pool, block_table), seqlens, scale,
+                  sel=sel, nthreads=nthreads, lib=lib)
+
+
+def kv_append_paged(k_pool, v_pool, k_new, v_new, block_table, pos):
+    """Return copies of the pools with key pos[b] of every (b, g) set to the new token: block
+    block_table[b, pos[b] // bs], row pos[b] % bs. A position outside [0, max_blocks * bs) or a
+    table entry outside [0, num_blocks) leaves the pools untouched."""
+    kp, vp = np.array(k_pool, copy=True), np.array(v_pool, copy=True)
+    nb, K, bs, _ = kp.shape
+    B, mb = np.asarray(block_table).shape
+    for b in range(B):
+        p = int(pos[b])
+        if not 0 <= p < mb * bs:
+            continue
+        blk = int(block_table[b][p // bs])
+        if 0 <= blk < nb:
+            kp[blk, :, p % bs, :] = k_new[b]
+            vp[blk, :, p % bs, :] = v_new[b]
+    return kp, vp

@@ -27,7 +27,7 @@ _LIB = os.path.join(_HERE, "libsynth.so")
 
 F32, BF16, F64 = 0, 1, 2
 SEED_BASE = 0x6A510000
-STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_KNEW, STREAM_VNEW = 1, 2, 3, 4, 5, 6
+STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_KNEW, STREAM_VNEW, STREAM_BLOCKS = 1, 2, 3, 4, 5, 6, 7
 
 
 def build(force: bool = False) -> str:
@@ -200,3 +200,73 @@ def prefill_inputs(w: PrefillShape) -> dict:
         "k": normal((w.B, w.S, w.K, w.d), w.dtype, w.seed, STREAM_K),
         "v": normal((w.B, w.S, w.K, w.d), w.dtype, w.seed, STREAM_V),
     }
+
+
+# --------------------------------------------------------------------------
+# paged caches: the same seeded cache values, scattered over a pool of blocks
+
+
+@dataclasses.dataclass(frozen=True)
+class PagedShape:
+    name: str
+    base: str          # the DecodeShape whose values are paged
+    block_size: int    # keys per block
+    spare_blocks: int  # pool blocks no sequence points to (NaN)
+
+
+PAGED_WORKLOADS = {
+    "paged_llama3_8b_decode_b8_h32_k8_d128_s8192_bs16": PagedShape(
+        "paged_llama3_8b_decode_b8_h32_k8_d128_s8192_bs16", "llama3_8b_decode_b8_h32_k8_d128_s8192", 16, 64),
+    "paged_ragged_70b_decode_b32_h64_k8_d128_s1k_16k_bs64": PagedShape(
+        "paged_ragged_70b_decode_b32_h64_k8_d128_s1k_16k_bs64", "ragged_70b_decode_b32_h64_k8_d128_s1k_16k", 64, 64),
+}
+
+
+def permutation(n: int, seed: int, stream: int) -> np.ndarray:
+    """A uniformly random permutation of 0..n-1 (Fisher-Yates over the counter stream)."""
+    key = stream_key(seed, stream)
+    perm = np.arange(n, dtype=np.int64)
+    for i in range(n - 1, 0, -1):
+        j = draw(key, i) % (i + 1)
+        perm[i], perm[j] = perm[j], perm[i]
+    return perm
+
+
+def page(k_cache: np.ndarray, v_cache: np.ndarray, lens: np.ndarray, block_size: int, spare_blocks: int,
+         seed: int, append_row: bool = False) -> dict:
+    """Scatter caches [B,K,S_max,d] into pools [num_blocks,K,block_size,d] at random physical blocks.
+
+    Sequence b gets ceil(n_b / block_size) blocks, n_b = lens[b] (+1 with ``append_row``: the block of
+    row lens[b] is mapped as well); its other table entries are -1. Pool blocks that no entry points to
+    hold NaN. Returns k_pool, v_pool, block_table [B, max_blocks] int32.
+    """
+    B, K, S_max, d = k_cache.shape
+    assert S_max % block_size == 0
+    mb = S_max // block_size
+    n = np.minimum(np.asarray(lens, dtype=np.int64) + (1 if append_row else 0), S_max)
+    need = (n + block_size - 1) // block_size
+    nb = int(need.sum()) + spare_blocks
+    perm = permutation(nb, seed, STREAM_BLOCKS)
+    table = np.full((B, mb), -1, dtype=np.int32)
+    nan = np.uint16(0x7FC0) if k_cache.dtype == np.uint16 else np.nan
+    k_pool = np.full((nb, K, block_size, d), nan, dtype=k_cache.dtype)
+    v_pool = np.full((nb, K, block_size, d), nan, dtype=v_cache.dtype)
+    nxt = 0
+    for b in range(B):
+        for i in range(int(need[b])):
+            blk = int(perm[nxt])
+            nxt += 1
+            table[b, i] = blk
+            k_pool[blk] = k_cache[b, :, i * block_size:(i + 1) * block_size, :]
+            v_pool[blk] = v_cache[b, :, i * block_size:(i + 1) * block_size, :]
+    return {"k_pool": k_pool, "v_pool": v_pool, "block_table": table}
+
+
+def paged_inputs(pw: PagedShape) -> dict:
+    """decode_inputs of the base workload, plus its caches paged (k_pool, v_pool, block_table)."""
+    w = DECODE_WORKLOADS[pw.base]
+    inp = decode_inputs(w)
+    lens = inp["pos"] if w.append else inp["seqlens"]
+    inp.update(page(inp["k_cache"], inp["v_cache"], lens, pw.block_size, pw.spare_blocks, w.seed,
+                    append_row=w.append))
+    return inp

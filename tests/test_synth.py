@@ -45,3 +45,40 @@ def test_uniform_int_range_and_workload_lengths():
     w = synth.DECODE_WORKLOADS["ragged_70b_decode_b32_h64_k8_d128_s1k_16k"]
     lens = synth.seqlens_for(w)
     assert lens.shape == (32,) and lens.min() >= 1024 and lens.max() <= 16384
+
+
+def test_permutation_is_a_seeded_permutation():
+    p1 = synth.permutation(257, synth.SEED_BASE + 9, synth.STREAM_BLOCKS)
+    p2 = synth.permutation(257, synth.SEED_BASE + 9, synth.STREAM_BLOCKS)
+    p3 = synth.permutation(257, synth.SEED_BASE + 10, synth.STREAM_BLOCKS)
+    assert np.array_equal(np.sort(p1), np.arange(257))
+    assert np.array_equal(p1, p2) and not np.array_equal(p1, p3)
+
+
+def test_page_scatters_every_valid_row_once():
+    B, K, S, d, bs = 3, 2, 64, 8, 16
+    lens = np.array([64, 5, 33], dtype=np.int32)
+    kc = synth.cache(B * K, S, d, synth.BF16, 123, synth.STREAM_K, lens, K).reshape(B, K, S, d)
+    vc = synth.cache(B * K, S, d, synth.BF16, 123, synth.STREAM_V, lens, K).reshape(B, K, S, d)
+    pg = synth.page(kc, vc, lens, bs, spare_blocks=4, seed=123)
+    table, kp = pg["block_table"], pg["k_pool"]
+    need = (lens + bs - 1) // bs
+    assert kp.shape == (int(need.sum()) + 4, K, bs, d) and table.shape == (B, S // bs)
+    used = table[table >= 0]
+    assert len(used) == need.sum() and len(np.unique(used)) == len(used)
+    for b in range(B):
+        assert (table[b, need[b]:] == -1).all()
+        for i in range(need[b]):
+            assert np.array_equal(kp[table[b, i]], kc[b, :, i * bs:(i + 1) * bs])
+            assert np.array_equal(pg["v_pool"][table[b, i]], vc[b, :, i * bs:(i + 1) * bs])
+    spare = np.setdiff1d(np.arange(kp.shape[0]), used)
+    assert len(spare) == 4 and (kp[spare] == 0x7FC0).all()
+
+
+def test_paged_inputs_map_the_append_row():
+    # the block of each appended row (pos = len - 1) is mapped
+    w = synth.DECODE_WORKLOADS["llama3_8b_decode_b8_h32_k8_d128_s8192"]
+    pos = synth.seqlens_for(w) - 1
+    kc = np.zeros((w.B, 1, w.S_max, 2), dtype=np.uint16)  # a tiny stand-in cache with the same lengths
+    pg = synth.page(kc, kc, pos, 16, 2, w.seed, append_row=True)
+    assert (pg["block_table"][np.arange(w.B), pos // 16] >= 0).all()
