@@ -290,6 +290,7 @@ def bench_ours(args, rank, world, local):
 DECODE_EXTRA = ["ragged_70b_decode_b32_h64_k8_d128_s1k_16k", "long_ctx_gqa_b1_h64_k8_d128_s131072",
                 "long_ctx_mqa_b1_h64_k1_d128_s131072"]
 PREFILL = "causal_prefill_b4_s4096_h32_k8_d128"
+PAGED_EXTRA = list(synth.PAGED_WORKLOADS)
 
 
 class L2Flush:
@@ -348,6 +349,11 @@ def extra_measurements(args, only=None):
                      "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "l2": "flushed (512 MiB write, then 512 MiB read)"}
         del q, kc, vc, out, ws, flush
         torch.cuda.empty_cache()
+    # paged caches: the same workloads' values over randomly placed blocks
+    for name in PAGED_EXTRA:
+        if only is not None and name != only:
+            continue
+        res[name] = paged_measurement(args, name, peaks, 20 if only is None else args.steps)
     if only is not None and only != PREFILL:
         return res
     # causal prefill with the KV-cache write: FLOPs over the causal pairs (j <= i) only
@@ -380,6 +386,62 @@ def extra_measurements(args, only=None):
     if gqa.gqa_get_last_error() != (0, 0):
         raise RuntimeError("device error in extra measurements")
     return res
+
+
+def paged_measurement(args, name, peaks, steps):
+    """gqa_decode_paged (gqa_decode_append_paged for a workload with an append) of one paged workload."""
+    import torch
+
+    from kv_cache_02_b200 import gqa
+
+    pw = synth.PAGED_WORKLOADS[name]
+    w = synth.DECODE_WORKLOADS[pw.base]
+    inp = synth.paged_inputs(pw)
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).cuda()
+
+    q, kp, vp, table = to_dev(inp["q"]), to_dev(inp["k_pool"]), to_dev(inp["v_pool"]), to_dev(inp["block_table"])
+    out = torch.empty_like(q)
+    wsb = gqa.gqa_decode_paged_workspace_bytes(w.B, w.H, w.K, w.d, pw.block_size, table.shape[1], 0)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+    scale = 1.0 / np.sqrt(w.d)
+    if w.append:
+        pos, kn, vn = to_dev(inp["pos"]), to_dev(inp["k_new"]), to_dev(inp["v_new"])
+        lens = inp["pos"].astype(np.int64) + 1
+
+        def call():
+            gqa.gqa_decode_append_paged(out, q, kp, vp, kn, vn, table, pos, scale, 0, ws)
+    else:
+        sl = to_dev(inp["seqlens"])
+        lens = inp["seqlens"].astype(np.int64)
+
+        def call():
+            gqa.gqa_decode_paged(out, q, kp, vp, table, sl, scale, 0, ws)
+    kv_bytes = int(lens.sum()) * w.K * w.d * 2 * 2
+    flush = L2Flush()
+    times = []
+    for it in range(args.warmup + steps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            times.append(a.elapsed_time(b))
+    if gqa.gqa_get_last_error() != (0, 0):
+        raise RuntimeError(f"device error in {name}")
+    ms = statistics.median(times)
+    gbs = kv_bytes / (ms * 1e-3) / 1e9
+    r = {"ms": round(ms, 5), "kv_bytes": kv_bytes, "GB/s": round(gbs, 1),
+         "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "block_size": pw.block_size,
+         "call": "gqa_decode_append_paged" if w.append else "gqa_decode_paged",
+         "l2": "flushed (512 MiB write, then 512 MiB read)"}
+    del q, kp, vp, table, out, ws, flush
+    torch.cuda.empty_cache()
+    return r
 
 
 def cpu_baseline(inp, scale, kv_bytes_layer):
@@ -436,7 +498,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads and the CPU baseline")
-    ap.add_argument("--only", choices=DECODE_EXTRA + [PREFILL], default=None,
+    ap.add_argument("--only", choices=DECODE_EXTRA + PAGED_EXTRA + [PREFILL], default=None,
                     help="time one other workload alone (for profiling); prints its own JSON, not the contract line")
     ap.add_argument("--layers", type=int, default=32,
                     help="layers per step (32 for the model; fewer only for small profiling captures)")

@@ -65,6 +65,8 @@ typedef enum {
 #define GQA_DEVERR_APPEND_POS 0x1u /* gqa_kv_append: pos[b] outside [0, S_max); row not written */
 #define GQA_DEVERR_SEQLEN 0x2u     /* gqa_decode: seqlens[b] outside [0, S_max]; out[b] set to zero */
 #define GQA_DEVERR_TIMEOUT 0x4u    /* a bounded wait in a pipelined kernel expired; output invalid */
+#define GQA_DEVERR_BLOCK 0x8u      /* paged cache: a block-table entry outside [0, num_blocks) was read;
+                                      block 0 was used in its place, output invalid */
 
 /*
  * gqa_kv_append - write one new token's K and V rows into the cache.
@@ -179,6 +181,53 @@ GQA_API int gqa_decode_append(void* out, const void* q, void* k_cache, void* v_c
 GQA_API int gqa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* seqlens, int B, int H, int K, int S_max, int d, float scale,
                                int num_splits, gqa_dtype dtype, gqa_stream_t stream);
+
+/*
+ * Paged KV cache: the paged forms of gqa_kv_append, gqa_decode and
+ * gqa_decode_append.
+ *
+ * "分組查詢注意力", section 下游 / 推論引擎與架構: a paged cache manages blocks
+ * of the K KV heads (not of the H query heads), and each block is broadcast
+ * to the H/K query heads of its group when it is used; "GQA 完全拆解",
+ * section 工程实现：权重布局、repeat 与 Kernel 融合: the block layout is organised
+ * by KV head and the kernel broadcasts within the group, and section
+ * 主流模型里的 GQA：KV 缓存账本: paging removes allocation fragmentation and is
+ * orthogonal to GQA. The pages give no block size or table format; here:
+ *
+ * k_pool, v_pool : [num_blocks, K, block_size, d]: block n holds block_size
+ *                  consecutive keys of one sequence for every KV head.
+ * block_table    : [B, max_blocks] int32, device. block_table[b, i] is the
+ *                  block holding keys i*block_size .. (i+1)*block_size - 1 of
+ *                  sequence b. Entries for keys a call does not touch are
+ *                  never read (they may hold anything, e.g. -1). An entry
+ *                  that is read and lies outside [0, num_blocks) sets
+ *                  GQA_DEVERR_BLOCK: the decode reads block 0 in its place
+ *                  (output invalid), the append writes nothing.
+ * block_size     : keys per block, a positive multiple of 16.
+ * max_blocks     : table row length; the capacity per sequence is
+ *                  S_max = max_blocks * block_size, and seqlens / pos are
+ *                  checked against it as for the contiguous cache.
+ *
+ * The results are those of the contiguous calls on the cache the table
+ * gathers: cache[b, g, t] = pool[block_table[b, t / block_size], g,
+ * t % block_size]. The decode forms are bf16 only (GQA_F32 returns
+ * GQA_ERR_UNSUPPORTED); the append takes bf16 or f32. The caller owns the
+ * pools, the table and the workspace. Invalid sizes return GQA_ERR_SHAPE.
+ */
+GQA_API size_t gqa_decode_paged_workspace_bytes(int B, int H, int K, int d, int block_size, int max_blocks,
+                                                int num_splits);
+GQA_API int gqa_decode_paged(void* out, const void* q, const void* k_pool, const void* v_pool,
+                             const int32_t* block_table, const int32_t* seqlens, int B, int H, int K, int d,
+                             int num_blocks, int block_size, int max_blocks, float scale, int num_splits,
+                             void* workspace, size_t workspace_bytes, gqa_dtype dtype, gqa_stream_t stream);
+GQA_API int gqa_decode_append_paged(void* out, const void* q, void* k_pool, void* v_pool, const void* k_new,
+                                    const void* v_new, const int32_t* block_table, const int32_t* pos, int B, int H,
+                                    int K, int d, int num_blocks, int block_size, int max_blocks, float scale,
+                                    int num_splits, void* workspace, size_t workspace_bytes, gqa_dtype dtype,
+                                    gqa_stream_t stream);
+GQA_API int gqa_kv_append_paged(void* k_pool, void* v_pool, const void* k_new, const void* v_new,
+                                const int32_t* block_table, const int32_t* pos, int B, int K, int d, int num_blocks,
+                                int block_size, int max_blocks, gqa_dtype dtype, gqa_stream_t stream);
 
 /*
  * gqa_prefill_causal - causal self-attention over a whole prompt, and the

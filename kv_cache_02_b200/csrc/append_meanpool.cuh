@@ -10,9 +10,15 @@ namespace gqa {
 // ---------------------------------------------------------------------------
 // gqa_kv_append: k_cache[b, g, pos[b], :] = k_new[b, g, :] (and V).
 // One thread per 16-byte chunk of a new row; both caches in one launch.
+// With a block table (gqa_kv_append_paged) the caches are pools of
+// num_blocks blocks [K, block_size, d], S_max = max_blocks * block_size, and
+// key pos[b] of sequence b is row pos[b] % block_size of block
+// block_table[b * max_blocks + pos[b] / block_size].
 __global__ void kv_append_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                                  const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
-                                 const int32_t* __restrict__ pos, int B, int K, int S_max, int chunks_per_row) {
+                                 const int32_t* __restrict__ pos, int B, int K, int S_max, int chunks_per_row,
+                                 const int32_t* __restrict__ block_table, int max_blocks, int block_size,
+                                 int num_blocks) {
   const long long per_tensor = (long long)B * K * chunks_per_row;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < 2 * per_tensor;
        i += (long long)gridDim.x * blockDim.x) {
@@ -20,13 +26,23 @@ __global__ void kv_append_kernel(uint4* __restrict__ k_cache, uint4* __restrict_
     const long long j = is_v ? i - per_tensor : i;
     const int c = (int)(j % chunks_per_row);
     const long long row = j / chunks_per_row;  // b * K + g
-    const int b = (int)(row / K);
+    const int b = (int)(row / K), g = (int)(row % K);
     const int p = __ldg(pos + b);
+    const bool reporter = c == 0 && !is_v && g == 0;  // one thread per sequence reports
     if (p < 0 || p >= S_max) {
-      if (c == 0 && !is_v && (row % K) == 0) raise_error(GQA_DEVERR_APPEND_POS);
+      if (reporter) raise_error(GQA_DEVERR_APPEND_POS);
       continue;
     }
-    const long long dst = (row * S_max + p) * chunks_per_row + c;
+    long long dst_row = row * S_max + p;
+    if (block_table != nullptr) {
+      const int blk = __ldg(block_table + (size_t)b * max_blocks + p / block_size);
+      if ((unsigned)blk >= (unsigned)num_blocks) {
+        if (reporter) raise_error(GQA_DEVERR_BLOCK);
+        continue;
+      }
+      dst_row = ((long long)blk * K + g) * block_size + p % block_size;
+    }
+    const long long dst = dst_row * chunks_per_row + c;
     if (is_v)
       v_cache[dst] = __ldg(v_new + j);
     else

@@ -73,6 +73,13 @@ struct DecodeParams {
   int nitems;                  // B * K * nsplit * hslices
   const int32_t* seqlens;
   int B, H, K, S_max, G, hslices, chunk, nsplit;
+  // paged cache (gqa_decode_paged): null for the contiguous cache
+  // [B, K, S_max, D]; otherwise the cache is a pool of num_blocks blocks
+  // [K, block_size, D] and block_table[b * max_blocks + i] is the block that
+  // holds keys i * block_size .. (i + 1) * block_size - 1 of sequence b
+  // (S_max = max_blocks * block_size). The TMA maps view either as rows of D.
+  const int32_t* block_table;
+  int max_blocks, block_size, num_blocks;
   unsigned long long tag;      // 40-bit, nonzero, different on every call
   float scale_log2;            // scale * log2(e)
 };
@@ -110,6 +117,27 @@ __device__ __forceinline__ int take_ticket(unsigned long long* cnt, unsigned lon
   return 0;
 }
 
+// Row of key t of KV head g in the [rows, D] view of a paged pool, key t
+// being in block blk (a table entry: outside [0, num_blocks) it sets
+// GQA_DEVERR_BLOCK and block 0 is used).
+__device__ __forceinline__ int paged_row(const DecodeParams& p, int blk, int g, int t) {
+  if ((unsigned)blk >= (unsigned)p.num_blocks) {
+    raise_error(GQA_DEVERR_BLOCK);
+    blk = 0;
+  }
+  return (blk * p.K + g) * p.block_size + t % p.block_size;
+}
+
+// Row of key t of unit (b, g) in the [rows, D] view of the cache (kPaged
+// false) or the pool. A table entry outside [0, num_blocks) sets
+// GQA_DEVERR_BLOCK and reads block 0. Paging is a template parameter of the
+// kernels, so the contiguous kernels carry none of the paged code.
+template <bool kPaged>
+__device__ __forceinline__ int kv_row(const DecodeParams& p, int b, int g, int t) {
+  if constexpr (!kPaged) return (b * p.K + g) * p.S_max + t;
+  return paged_row(p, __ldg(p.block_table + (size_t)b * p.max_blocks + t / p.block_size), g, t);
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -135,20 +163,79 @@ __device__ __forceinline__ void consumer_bar() {
 // pieces shared by the bf16 kernels
 
 // TMA loads of one tile (rows of K and V of one unit) into ring stage `s`.
+// TMA loads of one tile into a ring stage: a full tile as one 64-row box per
+// 128-byte column half (tm_*64), a partial one as 16-row boxes (tm_*16). The
+// 128-byte swizzle repeats every 8 rows, so both land in the same layout.
+// The producer is one thread; fewer, larger boxes keep it ahead of the ring.
 template <int D>
-__device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* full, const CUtensorMap* tm_k,
-                                           const CUtensorMap* tm_v, int row0, int rows, uint64_t policy) {
+__device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* full, const CUtensorMap* tm_k64,
+                                           const CUtensorMap* tm_v64, const CUtensorMap* tm_k16,
+                                           const CUtensorMap* tm_v16, int row0, int rows, uint64_t policy) {
   using C = DecCfg<D>;
+  if (rows == kDecTileKeys) {
+    mbar_arrive_expect_tx(full, (uint32_t)(kDecTileKeys * 128 * C::kHalves * 2));
+#pragma unroll
+    for (int hf = 0; hf < C::kHalves; ++hf) {
+      tma_load_2d(stage + hf * C::kHalfBytes, tm_k64, hf * 64, row0, full, policy);
+      tma_load_2d(stage + C::kTileBytes + hf * C::kHalfBytes, tm_v64, hf * 64, row0, full, policy);
+    }
+    return;
+  }
   const int nbox = (rows + kDecBoxRows - 1) / kDecBoxRows;
   mbar_arrive_expect_tx(full, (uint32_t)(nbox * kDecBoxRows * 128 * C::kHalves * 2));
   for (int bx = 0; bx < nbox; ++bx) {
 #pragma unroll
     for (int hf = 0; hf < C::kHalves; ++hf) {
       const int off = hf * C::kHalfBytes + bx * kDecBoxRows * 128;
-      tma_load_2d(stage + off, tm_k, hf * 64, row0 + bx * kDecBoxRows, full, policy);
-      tma_load_2d(stage + C::kTileBytes + off, tm_v, hf * 64, row0 + bx * kDecBoxRows, full, policy);
+      tma_load_2d(stage + off, tm_k16, hf * 64, row0 + bx * kDecBoxRows, full, policy);
+      tma_load_2d(stage + C::kTileBytes + off, tm_v16, hf * 64, row0 + bx * kDecBoxRows, full, policy);
     }
   }
+}
+
+// The same for a paged cache: a full tile inside one block (block size a
+// multiple of 64) as 64-row boxes, otherwise each 16-row box at its own row;
+// blk holds the table entries of the boxes' keys (tile_blocks), loaded a
+// tile ahead.
+template <int D>
+__device__ __forceinline__ void issue_tile_paged(uint8_t* stage, uint64_t* full, const CUtensorMap* tm_k64,
+                                                 const CUtensorMap* tm_v64, const CUtensorMap* tm_k16,
+                                                 const CUtensorMap* tm_v16, const DecodeParams& p, int g, int t0,
+                                                 const int (&blk)[kDecTileKeys / kDecBoxRows], int rows,
+                                                 uint64_t policy) {
+  using C = DecCfg<D>;
+  if (rows == kDecTileKeys && p.block_size % kDecTileKeys == 0) {
+    issue_tile<D>(stage, full, tm_k64, tm_v64, tm_k16, tm_v16, paged_row(p, blk[0], g, t0), rows, policy);
+    return;
+  }
+  int brow[kDecTileKeys / kDecBoxRows];
+#pragma unroll
+  for (int bx = 0; bx < kDecTileKeys / kDecBoxRows; ++bx)
+    brow[bx] = bx * kDecBoxRows < rows ? paged_row(p, blk[bx], g, t0 + bx * kDecBoxRows) : 0;
+  const int nbox = (rows + kDecBoxRows - 1) / kDecBoxRows;
+  mbar_arrive_expect_tx(full, (uint32_t)(nbox * kDecBoxRows * 128 * C::kHalves * 2));
+#pragma unroll
+  for (int bx = 0; bx < kDecTileKeys / kDecBoxRows; ++bx) {
+    if (bx >= nbox) break;
+#pragma unroll
+    for (int hf = 0; hf < C::kHalves; ++hf) {
+      const int off = hf * C::kHalfBytes + bx * kDecBoxRows * 128;
+      tma_load_2d(stage + off, tm_k16, hf * 64, brow[bx], full, policy);
+      tma_load_2d(stage + C::kTileBytes + off, tm_v16, hf * 64, brow[bx], full, policy);
+    }
+  }
+}
+
+// Table entries of the 16-row boxes of the tile of keys t0 .. t0 + rows - 1
+// of sequence b (every block size is a multiple of 16, so a box never
+// straddles blocks): independent loads, consumed only when the tile is
+// issued, so that they are in flight while the producer waits for a stage.
+__device__ __forceinline__ void tile_blocks(const DecodeParams& p, int b, int t0, int rows,
+                                            int (&blk)[kDecTileKeys / kDecBoxRows]) {
+  const int32_t* row = p.block_table + (size_t)b * p.max_blocks;
+#pragma unroll
+  for (int bx = 0; bx < kDecTileKeys / kDecBoxRows; ++bx)
+    blk[bx] = bx * kDecBoxRows < rows ? __ldg(row + (t0 + bx * kDecBoxRows) / p.block_size) : 0;
 }
 
 // Q^T as the B operand (k = dims, n = heads): lane holds head lane/4, dims
@@ -414,7 +501,7 @@ __device__ __forceinline__ void item_epilogue(const DecodeParams& p, const ItemC
 // tile just landed in shared memory (one warp, one 16-byte chunk per lane)
 // and are written to the cache at that row. The tile's rows are cache rows
 // t0 .. t0+rows-1, so row r is cache row len-1 = pos.
-template <int D>
+template <int D, bool kPaged>
 __device__ __forceinline__ void append_row(const DecodeParams& p, const ItemCoord& c, uint8_t* stage, int r,
                                            int lane) {
   using C = DecCfg<D>;
@@ -430,7 +517,7 @@ __device__ __forceinline__ void append_row(const DecodeParams& p, const ItemCoor
     *reinterpret_cast<uint4*>(dst) = val;
     if (c.hsl == 0) {  // one head slice writes the cache
       __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(is_v ? p.v_cache_w : p.k_cache_w);
-      reinterpret_cast<uint4*>(cache + (row * p.S_max + pos) * D)[ch] = val;
+      reinterpret_cast<uint4*>(cache + (size_t)kv_row<kPaged>(p, c.b, c.g, pos) * D)[ch] = val;
     }
   }
   // the stage is refilled by TMA (async proxy) once released: order these writes first
@@ -438,9 +525,10 @@ __device__ __forceinline__ void append_row(const DecodeParams& p, const ItemCoor
   __syncwarp();
 }
 
-template <int D>
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(kDecThreads, 2)
-    decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v64,
+                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const DecodeParams p) {
   using C = DecCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -469,6 +557,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   if (warp == kDecConsumerWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      prefetch_tensormap(&tm_k64);
+      prefetch_tensormap(&tm_v64);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
       const uint64_t policy = l2_policy_evict_first();
@@ -497,19 +587,31 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           continue;
         }
         const int ntiles = (t_end - t_begin + kDecTileKeys - 1) / kDecTileKeys;
-        const int row_base = c.unit * p.S_max;
+        int blk[kDecTileKeys / kDecBoxRows], blk_next[kDecTileKeys / kDecBoxRows];
+        if constexpr (kPaged) tile_blocks(p, c.b, t_begin, min(kDecTileKeys, t_end - t_begin), blk_next);
         for (int tt = 0; tt < ntiles && ok; ++tt, ++it) {
           const int s = it % C::kStages;
-          if (it >= C::kStages) ok = mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1);
-          if (!ok) break;
           const int t0 = t_begin + tt * kDecTileKeys;
           const int rows = min(kDecTileKeys, t_end - t0);
+          if constexpr (kPaged) {  // this tile's table entries; the next tile's load during the wait
+#pragma unroll
+            for (int bx = 0; bx < kDecTileKeys / kDecBoxRows; ++bx) blk[bx] = blk_next[bx];
+            if (tt + 1 < ntiles)
+              tile_blocks(p, c.b, t0 + kDecTileKeys, min(kDecTileKeys, t_end - t0 - kDecTileKeys), blk_next);
+          }
+          if (it >= C::kStages) ok = mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1);
+          if (!ok) break;
           const int new_row = (p.len_add && t0 <= len - 1 && len - 1 < t0 + rows) ? len - 1 - t0 : -1;
           info[s] = StageInfo{item, rows,
                               (tt == 0 ? kTileFirst : 0) | (tt == ntiles - 1 ? kTileLast : 0) |
                                   (len <= p.chunk ? kUnitSingleSplit : 0),
                               new_row};
-          issue_tile<D>(smem + s * C::kStageBytes, &full[s], &tm_k, &tm_v, row_base + t0, rows, policy);
+          if constexpr (kPaged)
+            issue_tile_paged<D>(smem + s * C::kStageBytes, &full[s], &tm_k64, &tm_v64, &tm_k, &tm_v, p, c.g, t0, blk,
+                                rows, policy);
+          else
+            issue_tile<D>(smem + s * C::kStageBytes, &full[s], &tm_k64, &tm_v64, &tm_k, &tm_v, c.unit * p.S_max + t0,
+                          rows, policy);
         }
         if (!ok) break;
       }
@@ -546,7 +648,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       st.reset();
     }
     if (si.new_row >= 0 && (si.new_row >> 4) == warp)
-      append_row<D>(p, cur, smem + s * C::kStageBytes, si.new_row, lane);
+      append_row<D, kPaged>(p, cur, smem + s * C::kStageBytes, si.new_row, lane);
     if (kb < si.rows) warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);

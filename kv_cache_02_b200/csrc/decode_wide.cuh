@@ -52,30 +52,78 @@ struct WideCfg {  // head dim 128
   static constexpr int kOCol = 256;  // O: columns [256, 384)
 };
 
-// TMA loads of `rows` keys of one unit: 64-row boxes, then 16-row boxes for the tail
+// The TMA boxes of the tile of `rows` keys from t0 of unit (b, g): 64-row
+// boxes where a 64-key group lies in one block (the contiguous cache, or
+// blocks of a multiple of 64 keys), otherwise 16-row boxes; 16-row boxes for
+// the tail. For a paged cache the boxes' table entries are loaded first
+// (wide_tile_blocks, a tile ahead) and turned into rows when the tile is
+// issued, so the loads are in flight while the producer waits for a stage.
+struct WideTileRows {
+  int n64, n16;
+  int r64[kWideKeys / kWideBox];
+  int r16[kWideKeys / kDecBoxRows];
+};
+
+template <bool kPaged>
+__device__ __forceinline__ void wide_tile_shape(const DecodeParams& p, int rows, WideTileRows& tr) {
+  const bool big = !kPaged || p.block_size % kWideBox == 0;
+  tr.n64 = big ? rows / kWideBox : 0;
+  tr.n16 = (rows - tr.n64 * kWideBox + kDecBoxRows - 1) / kDecBoxRows;
+}
+
+// paged: table entries of the boxes (r64 / r16 hold block numbers until wide_tile_rows)
+__device__ __forceinline__ void wide_tile_blocks(const DecodeParams& p, int b, int t0, WideTileRows& tr) {
+  const int32_t* row = p.block_table + (size_t)b * p.max_blocks;
+#pragma unroll
+  for (int bx = 0; bx < kWideKeys / kWideBox; ++bx)
+    tr.r64[bx] = bx < tr.n64 ? __ldg(row + (t0 + bx * kWideBox) / p.block_size) : 0;
+#pragma unroll
+  for (int bx = 0; bx < kWideKeys / kDecBoxRows; ++bx)
+    tr.r16[bx] = bx < tr.n16 ? __ldg(row + (t0 + tr.n64 * kWideBox + bx * kDecBoxRows) / p.block_size) : 0;
+}
+
+template <bool kPaged>
+__device__ __forceinline__ void wide_tile_rows(const DecodeParams& p, int b, int g, int t0, WideTileRows& tr) {
+#pragma unroll
+  for (int bx = 0; bx < kWideKeys / kWideBox; ++bx) {
+    if (bx >= tr.n64) break;
+    const int t = t0 + bx * kWideBox;
+    tr.r64[bx] = kPaged ? paged_row(p, tr.r64[bx], g, t) : kv_row<false>(p, b, g, t);
+  }
+#pragma unroll
+  for (int bx = 0; bx < kWideKeys / kDecBoxRows; ++bx) {
+    if (bx >= tr.n16) break;
+    const int t = t0 + tr.n64 * kWideBox + bx * kDecBoxRows;
+    tr.r16[bx] = kPaged ? paged_row(p, tr.r16[bx], g, t) : kv_row<false>(p, b, g, t);
+  }
+}
+
 __device__ __forceinline__ void wide_issue_tile(uint8_t* stage, uint64_t* full, const CUtensorMap* tm_k64,
                                                 const CUtensorMap* tm_v64, const CUtensorMap* tm_k16,
-                                                const CUtensorMap* tm_v16, int row0, int rows, uint64_t policy) {
+                                                const CUtensorMap* tm_v16, const WideTileRows& tr, uint64_t policy) {
   using C = WideCfg;
-  const int n64 = rows / kWideBox;
-  const int rem = rows - n64 * kWideBox;
-  const int n16 = (rem + kDecBoxRows - 1) / kDecBoxRows;
-  mbar_arrive_expect_tx(full, (uint32_t)((n64 * kWideBox + n16 * kDecBoxRows) * 128 * 2 * 2));
-  for (int bx = 0; bx < n64; ++bx)
+  mbar_arrive_expect_tx(full, (uint32_t)((tr.n64 * kWideBox + tr.n16 * kDecBoxRows) * 128 * 2 * 2));
+#pragma unroll
+  for (int bx = 0; bx < kWideKeys / kWideBox; ++bx) {
+    if (bx >= tr.n64) break;
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int off = hf * C::kHalf + bx * kWideBox * 128;
-      tma_load_2d(stage + off, tm_k64, hf * 64, row0 + bx * kWideBox, full, policy);
-      tma_load_2d(stage + C::kTile + off, tm_v64, hf * 64, row0 + bx * kWideBox, full, policy);
+      tma_load_2d(stage + off, tm_k64, hf * 64, tr.r64[bx], full, policy);
+      tma_load_2d(stage + C::kTile + off, tm_v64, hf * 64, tr.r64[bx], full, policy);
     }
-  for (int bx = 0; bx < n16; ++bx)
+  }
+#pragma unroll
+  for (int bx = 0; bx < kWideKeys / kDecBoxRows; ++bx) {
+    if (bx >= tr.n16) break;
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const int r = n64 * kWideBox + bx * kDecBoxRows;
+      const int r = tr.n64 * kWideBox + bx * kDecBoxRows;
       const int off = hf * C::kHalf + r * 128;
-      tma_load_2d(stage + off, tm_k16, hf * 64, row0 + r, full, policy);
-      tma_load_2d(stage + C::kTile + off, tm_v16, hf * 64, row0 + r, full, policy);
+      tma_load_2d(stage + off, tm_k16, hf * 64, tr.r16[bx], full, policy);
+      tma_load_2d(stage + C::kTile + off, tm_v16, hf * 64, tr.r16[bx], full, policy);
     }
+  }
 }
 
 // One tile of the online softmax for the two heads a thread holds. x: the raw
@@ -156,6 +204,7 @@ __device__ __forceinline__ void wide_softmax_tile(float (&x)[64], int rows, int 
   l_b = l_b * alpha_b + sb;
 }
 
+template <bool kPaged>
 __global__ void __launch_bounds__(kWideThreads, 1)
     decode_wide_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k64,
                        const __grid_constant__ CUtensorMap tm_v64, const __grid_constant__ CUtensorMap tm_k16,
@@ -251,19 +300,27 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           tma_load_2d(smem + C::kQOff + hf * C::kQHalf, &tm_q, hf * 64, c.b * p.H + c.h0, q_full, q_policy);
         ++nq;
         const int ntiles = (t_end - t_begin + kWideKeys - 1) / kWideKeys;
-        const int row_base = c.unit * p.S_max;
+        WideTileRows tr_next;
+        wide_tile_shape<kPaged>(p, min(kWideKeys, t_end - t_begin), tr_next);
+        if constexpr (kPaged) wide_tile_blocks(p, c.b, t_begin, tr_next);
         for (int tt = 0; tt < ntiles && ok; ++tt, ++it) {
           const int s = it % C::kStages;
-          if (it >= C::kStages) ok = mbar_wait_bounded(&kv_empty[s], ((it / C::kStages) - 1) & 1);
-          if (!ok) break;
           const int t0 = t_begin + tt * kWideKeys;
           const int rows = min(kWideKeys, t_end - t0);
+          WideTileRows tr = tr_next;
+          if (tt + 1 < ntiles) {  // a paged cache's next table entries load during the wait
+            wide_tile_shape<kPaged>(p, min(kWideKeys, t_end - t0 - kWideKeys), tr_next);
+            if constexpr (kPaged) wide_tile_blocks(p, c.b, t0 + kWideKeys, tr_next);
+          }
+          if (it >= C::kStages) ok = mbar_wait_bounded(&kv_empty[s], ((it / C::kStages) - 1) & 1);
+          if (!ok) break;
+          wide_tile_rows<kPaged>(p, c.b, c.g, t0, tr);
           info[s] = StageInfo{item, rows,
                               (tt == 0 ? kTileFirst : 0) | (tt == ntiles - 1 ? kTileLast : 0) |
                                   (len <= p.chunk ? kUnitSingleSplit : 0),
                               -1};
-          wide_issue_tile(smem + C::kKVOff + s * C::kStage, &kv_full[s], &tm_k64, &tm_v64, &tm_k16, &tm_v16,
-                          row_base + t0, rows, policy);
+          wide_issue_tile(smem + C::kKVOff + s * C::kStage, &kv_full[s], &tm_k64, &tm_v64, &tm_k16, &tm_v16, tr,
+                          policy);
         }
         if (!ok) break;
       }

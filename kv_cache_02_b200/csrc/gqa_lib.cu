@@ -111,12 +111,28 @@ unsigned long long next_call_tag() {
   return t ? t : 1ull;
 }
 
-bool valid_decode_shape(int B, int H, int K, int S_max, int d) {
+bool valid_decode_shape(int B, int H, int K, int S_max, int d, bool paged = false) {
   if (B < 0 || H <= 0 || K <= 0 || S_max <= 0) return false;
   if (H % K != 0) return false;
   if (d != 64 && d != 128) return false;
-  if ((long long)B * K * S_max >= (1ll << 31)) return false;  // TMA row coordinate is int32
+  if (!paged && (long long)B * K * S_max >= (1ll << 31)) return false;  // TMA row coordinate is int32
   if ((long long)B * H >= (1ll << 31)) return false;
+  return true;
+}
+
+// A paged cache: a pool of num_blocks blocks [K, block_size, d] and a block
+// table [B, max_blocks] (see DecodeParams).
+struct PagedCache {
+  const int32_t* table = nullptr;
+  int num_blocks = 0, block_size = 0, max_blocks = 0;
+};
+
+bool valid_paged(const PagedCache& pc, int B, int K) {
+  if (pc.num_blocks <= 0 || pc.block_size <= 0 || pc.max_blocks <= 0) return false;
+  if (pc.block_size % 16 != 0) return false;  // a 16-row TMA box never straddles blocks
+  if ((long long)pc.max_blocks * pc.block_size >= (1ll << 31)) return false;
+  if ((long long)pc.num_blocks * K * pc.block_size >= (1ll << 31)) return false;  // TMA row coordinate
+  if ((long long)B * pc.max_blocks >= (1ll << 31)) return false;
   return true;
 }
 
@@ -128,9 +144,11 @@ int decode_ctas_per_sm(int dev) {
   if (cache[dev] == 0) {
     int n = 0;
     using C = gqa::DecCfg<D>;
-    if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_bf16_kernel<D>, gqa::kDecThreads,
+        cudaFuncSetAttribute(gqa::decode_bf16_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_bf16_kernel<D, false>, gqa::kDecThreads,
                                                       C::kSmemBytes) != cudaSuccess ||
         n <= 0) {
       cudaGetLastError();  // no GPU here: plan with the B200 figure
@@ -147,9 +165,11 @@ int wide_ctas_per_sm(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return 1;
   if (cache[dev] == 0) {
     int n = 0;
-    if (cudaFuncSetAttribute(gqa::decode_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gqa::decode_wide_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gqa::WideCfg::kSmemBytes) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_wide_kernel, gqa::kWideThreads,
+        cudaFuncSetAttribute(gqa::decode_wide_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gqa::WideCfg::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_wide_kernel<false>, gqa::kWideThreads,
                                                       gqa::WideCfg::kSmemBytes) != cudaSuccess ||
         n <= 0) {
       cudaGetLastError();
@@ -209,31 +229,41 @@ DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gq
   return pl;
 }
 
+// rows: of the [rows, D] view of the cache (B * K * S_max) or the pool (num_blocks * K * block_size)
 template <int D>
-int launch_decode_bf16(const DecodePlan& pl, const DecodeParams& p, const void* kc, const void* vc, int B, int K,
-                       int S_max, cudaStream_t st) {
-  CUtensorMap tk, tv;
-  const uint64_t rows = (uint64_t)B * K * S_max;
-  if (!encode_rows_bf16(&tk, kc, rows, D, gqa::kDecBoxRows) || !encode_rows_bf16(&tv, vc, rows, D, gqa::kDecBoxRows))
+int launch_decode_bf16(const DecodePlan& pl, const DecodeParams& p, const void* kc, const void* vc, uint64_t rows,
+                       cudaStream_t st) {
+  CUtensorMap tk64, tv64, tk, tv;  // 64-row boxes for full tiles, 16-row boxes for the rest
+  if (!encode_rows_bf16(&tk64, kc, rows, D, gqa::kDecTileKeys) ||
+      !encode_rows_bf16(&tv64, vc, rows, D, gqa::kDecTileKeys) ||
+      !encode_rows_bf16(&tk, kc, rows, D, gqa::kDecBoxRows) || !encode_rows_bf16(&tv, vc, rows, D, gqa::kDecBoxRows))
     return GQA_ERR_CUDA;
   using C = gqa::DecCfg<D>;
   decode_ctas_per_sm<D>(current_device());  // sets the shared-memory attribute once per device
-  gqa::decode_bf16_kernel<D><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(tk, tv, p);
+  if (p.block_table)
+    gqa::decode_bf16_kernel<D, true><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(tk64, tv64, tk, tv,
+                                                                                                p);
+  else
+    gqa::decode_bf16_kernel<D, false><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(tk64, tv64, tk, tv,
+                                                                                                 p);
   return launch_status();
 }
 
 int launch_decode_wide(const DecodePlan& pl, const DecodeParams& p, const void* q, const void* kc, const void* vc,
-                       int B, int H, int K, int S_max, cudaStream_t st) {
+                       int B, int H, uint64_t rows, cudaStream_t st) {
   CUtensorMap tq, tk64, tv64, tk16, tv16;
-  const uint64_t rows = (uint64_t)B * K * S_max;
   if (!encode_rows_bf16(&tq, q, (uint64_t)B * H, 128, gqa::kWideHeads) ||
       !encode_rows_bf16(&tk64, kc, rows, 128, gqa::kWideBox) || !encode_rows_bf16(&tv64, vc, rows, 128, gqa::kWideBox) ||
       !encode_rows_bf16(&tk16, kc, rows, 128, gqa::kDecBoxRows) ||
       !encode_rows_bf16(&tv16, vc, rows, 128, gqa::kDecBoxRows))
     return GQA_ERR_CUDA;
   wide_ctas_per_sm(current_device());  // sets the shared-memory attribute once per device
-  gqa::decode_wide_kernel<<<(unsigned)pl.grid, gqa::kWideThreads, gqa::WideCfg::kSmemBytes, st>>>(tq, tk64, tv64,
-                                                                                                 tk16, tv16, p);
+  if (p.block_table)
+    gqa::decode_wide_kernel<true><<<(unsigned)pl.grid, gqa::kWideThreads, gqa::WideCfg::kSmemBytes, st>>>(
+        tq, tk64, tv64, tk16, tv16, p);
+  else
+    gqa::decode_wide_kernel<false><<<(unsigned)pl.grid, gqa::kWideThreads, gqa::WideCfg::kSmemBytes, st>>>(
+        tq, tk64, tv64, tk16, tv16, p);
   return launch_status();
 }
 
@@ -291,25 +321,6 @@ const char* gqa_status_string(int status) {
     case GQA_ERR_SCRATCH_LIMIT: return "GQA_ERR_SCRATCH_LIMIT";
     default: return "GQA_ERR_UNKNOWN";
   }
-}
-
-int gqa_kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* pos, int B,
-                  int K, int S_max, int d, gqa_dtype dtype, gqa_stream_t stream) {
-  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
-  if (B < 0 || K <= 0 || S_max <= 0) return GQA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return GQA_ERR_SHAPE;
-  if (B == 0) return GQA_OK;
-  if (!k_cache || !v_cache || !k_new || !v_new || !pos) return GQA_ERR_INVALID_ARG;
-  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new)) return GQA_ERR_ALIGN;
-  const int elt = dtype == GQA_F32 ? 4 : 2;
-  const int cpr = d * elt / 16;
-  const long long work = 2ll * B * K * cpr;
-  const int dev = current_device();
-  const int grid = grid_for(work, 256, sm_count(dev));
-  gqa::kv_append_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k_new),
-      static_cast<const uint4*>(v_new), pos, B, K, S_max, cpr);
-  return launch_status();
 }
 
 size_t gqa_decode_workspace_bytes(int B, int H, int K, int S_max, int d, int num_splits) {
@@ -370,15 +381,40 @@ cudaError_t launch_combine(void* out, const DecodeParams& p, const int32_t* seql
                                                 units, st);
 }
 
-// gqa_decode, and with append != 0 gqa_decode_append (seqlens then holds pos).
+// gqa_kv_append, and with a paged cache gqa_kv_append_paged (S_max = max_blocks * block_size).
+int kv_append_impl(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* pos, int B,
+                   int K, int S_max, int d, gqa_dtype dtype, gqa_stream_t stream, const PagedCache* pc) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (B < 0 || K <= 0 || S_max <= 0) return GQA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return GQA_ERR_SHAPE;
+  if (B == 0) return GQA_OK;
+  if (!k_cache || !v_cache || !k_new || !v_new || !pos) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new)) return GQA_ERR_ALIGN;
+  const int elt = dtype == GQA_F32 ? 4 : 2;
+  const int cpr = d * elt / 16;
+  const long long work = 2ll * B * K * cpr;
+  const int dev = current_device();
+  const int grid = grid_for(work, 256, sm_count(dev));
+  gqa::kv_append_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k_new),
+      static_cast<const uint4*>(v_new), pos, B, K, S_max, cpr, pc ? pc->table : nullptr, pc ? pc->max_blocks : 0,
+      pc ? pc->block_size : 0, pc ? pc->num_blocks : 0);
+  return launch_status();
+}
+
+// gqa_decode, and with append != 0 gqa_decode_append (seqlens then holds pos);
+// with a paged cache (pc != null) their paged forms, S_max = max_blocks * block_size.
 int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
                 int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
-                gqa_dtype dtype, gqa_stream_t stream, const void* k_new, const void* v_new, int append) {
+                gqa_dtype dtype, gqa_stream_t stream, const void* k_new, const void* v_new, int append,
+                const PagedCache* pc = nullptr) {
   if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
   if (num_splits < 0 || B < 0 || H <= 0 || K <= 0 || S_max <= 0) return GQA_ERR_INVALID_ARG;
-  if (!valid_decode_shape(B, H, K, S_max, d)) return GQA_ERR_SHAPE;
+  if (!valid_decode_shape(B, H, K, S_max, d, pc != nullptr)) return GQA_ERR_SHAPE;
+  if (pc && !valid_paged(*pc, B, K)) return GQA_ERR_SHAPE;
+  if (pc && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;  // the paged forms stream bf16 by TMA
   if (B == 0) return GQA_OK;
-  if (!out || !q || !k_cache || !v_cache || !seqlens) return GQA_ERR_INVALID_ARG;
+  if (!out || !q || !k_cache || !v_cache || !seqlens || (pc && !pc->table)) return GQA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return GQA_ERR_ALIGN;
   if (append && (!k_new || !v_new)) return GQA_ERR_INVALID_ARG;
   if (append && (!aligned16(k_new) || !aligned16(v_new))) return GQA_ERR_ALIGN;
@@ -392,8 +428,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   const int G = H / K;
   cudaStream_t st = (cudaStream_t)stream;
   if (append && (dtype != GQA_BF16 || pl.wide)) {  // the append as its own launch, then the decode
-    const int rc = gqa_kv_append(const_cast<void*>(k_cache), const_cast<void*>(v_cache), k_new, v_new, seqlens, B, K,
-                                 S_max, d, dtype, stream);
+    const int rc = kv_append_impl(const_cast<void*>(k_cache), const_cast<void*>(v_cache), k_new, v_new, seqlens, B,
+                                  K, S_max, d, dtype, stream, pc);
     if (rc != GQA_OK) return rc;
   }
   DecodeParams p;
@@ -422,12 +458,17 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.chunk = pl.chunk;
   p.nsplit = pl.nsplit;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.block_table = pc ? pc->table : nullptr;
+  p.max_blocks = pc ? pc->max_blocks : 0;
+  p.block_size = pc ? pc->block_size : 0;
+  p.num_blocks = pc ? pc->num_blocks : 0;
+  const uint64_t rows = pc ? (uint64_t)pc->num_blocks * K * pc->block_size : (uint64_t)B * K * S_max;
   int rc;
   if (pl.wide)
-    rc = launch_decode_wide(pl, p, q, k_cache, v_cache, B, H, K, S_max, st);
+    rc = launch_decode_wide(pl, p, q, k_cache, v_cache, B, H, rows, st);
   else if (dtype == GQA_BF16)
-    rc = d == 128 ? launch_decode_bf16<128>(pl, p, k_cache, v_cache, B, K, S_max, st)
-                  : launch_decode_bf16<64>(pl, p, k_cache, v_cache, B, K, S_max, st);
+    rc = d == 128 ? launch_decode_bf16<128>(pl, p, k_cache, v_cache, rows, st)
+                  : launch_decode_bf16<64>(pl, p, k_cache, v_cache, rows, st);
   else
     rc = d == 128 ? launch_decode_f32<128>(pl, p, k_cache, v_cache, st)
                   : launch_decode_f32<64>(pl, p, k_cache, v_cache, st);
@@ -449,6 +490,25 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
 
 extern "C" {
 
+int gqa_kv_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new, const int32_t* pos, int B,
+                  int K, int S_max, int d, gqa_dtype dtype, gqa_stream_t stream) {
+  return kv_append_impl(k_cache, v_cache, k_new, v_new, pos, B, K, S_max, d, dtype, stream, nullptr);
+}
+
+int gqa_kv_append_paged(void* k_pool, void* v_pool, const void* k_new, const void* v_new, const int32_t* block_table,
+                        const int32_t* pos, int B, int K, int d, int num_blocks, int block_size, int max_blocks,
+                        gqa_dtype dtype, gqa_stream_t stream) {
+  PagedCache pc;
+  pc.table = block_table;
+  pc.num_blocks = num_blocks;
+  pc.block_size = block_size;
+  pc.max_blocks = max_blocks;
+  if (B < 0 || K <= 0) return GQA_ERR_INVALID_ARG;
+  if (!valid_paged(pc, B, K)) return GQA_ERR_SHAPE;
+  if (B > 0 && !block_table) return GQA_ERR_INVALID_ARG;
+  return kv_append_impl(k_pool, v_pool, k_new, v_new, pos, B, K, max_blocks * block_size, d, dtype, stream, &pc);
+}
+
 int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
                int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
                gqa_dtype dtype, gqa_stream_t stream) {
@@ -461,6 +521,45 @@ int gqa_decode_append(void* out, const void* q, void* k_cache, void* v_cache, co
                       void* workspace, size_t workspace_bytes, gqa_dtype dtype, gqa_stream_t stream) {
   return decode_impl(out, q, k_cache, v_cache, pos, B, H, K, S_max, d, scale, num_splits, workspace, workspace_bytes,
                      dtype, stream, k_new, v_new, 1);
+}
+
+int gqa_decode_paged(void* out, const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,
+                     const int32_t* seqlens, int B, int H, int K, int d, int num_blocks, int block_size,
+                     int max_blocks, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                     gqa_dtype dtype, gqa_stream_t stream) {
+  PagedCache pc;
+  pc.table = block_table;
+  pc.num_blocks = num_blocks;
+  pc.block_size = block_size;
+  pc.max_blocks = max_blocks;
+  if (block_size <= 0 || max_blocks <= 0 || (long long)max_blocks * block_size >= (1ll << 31)) return GQA_ERR_SHAPE;
+  return decode_impl(out, q, k_pool, v_pool, seqlens, B, H, K, max_blocks * block_size, d, scale, num_splits,
+                     workspace, workspace_bytes, dtype, stream, nullptr, nullptr, 0, &pc);
+}
+
+int gqa_decode_append_paged(void* out, const void* q, void* k_pool, void* v_pool, const void* k_new,
+                            const void* v_new, const int32_t* block_table, const int32_t* pos, int B, int H, int K,
+                            int d, int num_blocks, int block_size, int max_blocks, float scale, int num_splits,
+                            void* workspace, size_t workspace_bytes, gqa_dtype dtype, gqa_stream_t stream) {
+  PagedCache pc;
+  pc.table = block_table;
+  pc.num_blocks = num_blocks;
+  pc.block_size = block_size;
+  pc.max_blocks = max_blocks;
+  if (block_size <= 0 || max_blocks <= 0 || (long long)max_blocks * block_size >= (1ll << 31)) return GQA_ERR_SHAPE;
+  return decode_impl(out, q, k_pool, v_pool, pos, B, H, K, max_blocks * block_size, d, scale, num_splits, workspace,
+                     workspace_bytes, dtype, stream, k_new, v_new, 1, &pc);
+}
+
+size_t gqa_decode_paged_workspace_bytes(int B, int H, int K, int d, int block_size, int max_blocks, int num_splits) {
+  if (block_size <= 0 || block_size % 16 != 0 || max_blocks <= 0 ||
+      (long long)max_blocks * block_size >= (1ll << 31))
+    return 0;
+  const int S_max = max_blocks * block_size;
+  if (!valid_decode_shape(B, H, K, S_max, d, true) || num_splits < 0) return 0;
+  const DecodePlan a = plan_decode(B, H, K, S_max, d, num_splits, GQA_BF16, sm_count(current_device()));
+  if (a.ws_bytes == (size_t)-1) return 0;
+  return a.ws_bytes;
 }
 
 int gqa_prefill_causal(void* out, const void* q, const void* k, const void* v, void* k_cache, void* v_cache, int B,

@@ -22,12 +22,13 @@ GQA_F32, GQA_BF16 = 0, 1
 GQA_OK = 0
 GQA_ERR_DEVICE = -5
 GQA_ERR_UNSUPPORTED = -6
-GQA_DEVERR_APPEND_POS, GQA_DEVERR_SEQLEN, GQA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
+GQA_DEVERR_APPEND_POS, GQA_DEVERR_SEQLEN, GQA_DEVERR_TIMEOUT, GQA_DEVERR_BLOCK = 0x1, 0x2, 0x4, 0x8
 
 GQA_ERR_SCRATCH_LIMIT = -7
 GQA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode", "gqa_decode_append", "gqa_decode_noalloc",
+            "gqa_decode_paged_workspace_bytes", "gqa_decode_paged", "gqa_decode_append_paged", "gqa_kv_append_paged",
             "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string")
 
 
@@ -53,6 +54,14 @@ def _load():
     lib.gqa_decode_append.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, I, P]
     lib.gqa_decode_noalloc.restype = I
     lib.gqa_decode_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, I, P]
+    lib.gqa_decode_paged_workspace_bytes.restype = SZ
+    lib.gqa_decode_paged_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+    lib.gqa_decode_paged.restype = I
+    lib.gqa_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P, SZ, I, P]
+    lib.gqa_decode_append_paged.restype = I
+    lib.gqa_decode_append_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P, SZ, I, P]
+    lib.gqa_kv_append_paged.restype = I
+    lib.gqa_kv_append_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P]
     lib.gqa_prefill_causal.restype = I
     lib.gqa_prefill_causal.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gqa_meanpool_kv.restype = I
@@ -157,6 +166,57 @@ def gqa_decode_noalloc(out, q, k_cache, v_cache, seqlens, scale: float, num_spli
     _check("gqa_decode_noalloc", _lib.gqa_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                                          _ptr(seqlens), B, H, K, S_max, d, float(scale),
                                                          int(num_splits), _dtype(q), _stream(stream)))
+
+
+def gqa_decode_paged_workspace_bytes(B: int, H: int, K: int, d: int, block_size: int, max_blocks: int,
+                                     num_splits: int = 0) -> int:
+    return int(_lib.gqa_decode_paged_workspace_bytes(B, H, K, d, block_size, max_blocks, num_splits))
+
+
+def _paged_shapes(q, k_pool, v_pool, block_table):
+    B, H, d = q.shape
+    num_blocks, K, block_size, dk = k_pool.shape
+    assert dk == d and v_pool.shape == k_pool.shape
+    assert block_table.dtype == torch.int32 and block_table.dim() == 2 and block_table.shape[0] == B
+    return B, H, K, d, num_blocks, block_size, block_table.shape[1]
+
+
+def gqa_decode_paged(out, q, k_pool, v_pool, block_table, seqlens, scale: float, num_splits: int = 0,
+                     workspace=None, stream=None) -> None:
+    """out/q [B,H,d], pools [num_blocks,K,block_size,d], block_table [B,max_blocks] int32, seqlens [B] int32."""
+    B, H, K, d, nb, bs, mb = _paged_shapes(q, k_pool, v_pool, block_table)
+    assert out.shape == q.shape and seqlens.dtype == torch.int32 and seqlens.shape == (B,)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("gqa_decode_paged", _lib.gqa_decode_paged(_ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                                     _ptr(block_table), _ptr(seqlens), B, H, K, d, nb, bs, mb,
+                                                     float(scale), int(num_splits), _ptr(workspace), ws_bytes,
+                                                     _dtype(q), _stream(stream)))
+
+
+def gqa_decode_append_paged(out, q, k_pool, v_pool, k_new, v_new, block_table, pos, scale: float,
+                            num_splits: int = 0, workspace=None, stream=None) -> None:
+    """Append k_new/v_new [B,K,d] at key pos[b] of the paged cache, then decode over pos[b] + 1 keys."""
+    B, H, K, d, nb, bs, mb = _paged_shapes(q, k_pool, v_pool, block_table)
+    assert out.shape == q.shape and k_new.shape == (B, K, d) and v_new.shape == (B, K, d)
+    assert pos.dtype == torch.int32 and pos.shape == (B,)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("gqa_decode_append_paged",
+           _lib.gqa_decode_append_paged(_ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(k_new), _ptr(v_new),
+                                        _ptr(block_table), _ptr(pos), B, H, K, d, nb, bs, mb, float(scale),
+                                        int(num_splits), _ptr(workspace), ws_bytes, _dtype(q), _stream(stream)))
+
+
+def gqa_kv_append_paged(k_pool, v_pool, k_new, v_new, block_table, pos, stream=None) -> None:
+    """pools [num_blocks,K,block_size,d] (in place), k_new/v_new [B,K,d], block_table [B,max_blocks], pos [B]."""
+    num_blocks, K, block_size, d = k_pool.shape
+    B = k_new.shape[0]
+    assert v_pool.shape == k_pool.shape and k_new.shape == (B, K, d) and v_new.shape == (B, K, d)
+    assert block_table.dtype == torch.int32 and block_table.dim() == 2 and block_table.shape[0] == B
+    assert pos.dtype == torch.int32 and pos.shape == (B,)
+    _check("gqa_kv_append_paged",
+           _lib.gqa_kv_append_paged(_ptr(k_pool), _ptr(v_pool), _ptr(k_new), _ptr(v_new), _ptr(block_table),
+                                    _ptr(pos), B, K, d, num_blocks, block_size, block_table.shape[1],
+                                    _dtype(k_pool), _stream(stream)))
 
 
 def gqa_prefill_causal(out, q, k, v, scale: float, k_cache=None, v_cache=None, stream=None) -> None:

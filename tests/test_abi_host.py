@@ -28,7 +28,9 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     assert declared_symbols() == sorted(["gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode",
-                                         "gqa_decode_append", "gqa_decode_noalloc", "gqa_prefill_causal",
+                                         "gqa_decode_append", "gqa_decode_noalloc",
+                                         "gqa_decode_paged_workspace_bytes", "gqa_decode_paged",
+                                         "gqa_decode_append_paged", "gqa_kv_append_paged", "gqa_prefill_causal",
                                          "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string"])
 
 
@@ -83,6 +85,36 @@ def test_append_and_meanpool_reject_bad_arguments(lib):
     assert lib.gqa_meanpool_kv(P, P, 1, 6, 4, 64, 1, None) == -2
     assert lib.gqa_meanpool_kv(P, P, -1, 8, 4, 64, 1, None) == -1
     assert lib.gqa_meanpool_kv(None, None, 0, 8, 4, 64, 1, None) == 0
+
+
+def test_paged_calls_reject_bad_arguments(lib):
+    f = lib.gqa_decode_paged
+    # out, q, k_pool, v_pool, table, seqlens, B, H, K, d, num_blocks, block_size, max_blocks, scale, splits, ws, ws_bytes,
+    # dtype, stream
+    assert f(P, P, P, P, P, P, 2, 8, 2, 64, 64, 24, 8, 1.0, 0, None, 0, 1, None) == -2     # block size not 16k
+    assert f(P, P, P, P, P, P, 2, 8, 2, 64, 64, 0, 8, 1.0, 0, None, 0, 1, None) == -2
+    assert f(P, P, P, P, P, P, 2, 8, 2, 64, 64, 16, 0, 1.0, 0, None, 0, 1, None) == -2      # no table columns
+    assert f(P, P, P, P, P, P, 2, 6, 4, 64, 64, 16, 8, 1.0, 0, None, 0, 1, None) == -2      # H % K != 0
+    assert f(P, P, P, P, P, P, 2, 8, 2, 64, 64, 16, 8, 1.0, 0, None, 0, 0, None) == -6      # f32
+    assert f(P, P, P, P, None, P, 2, 8, 2, 64, 64, 16, 8, 1.0, 0, None, 0, 1, None) == -1   # no table
+    assert f(P, P, P + 4, P, P, P, 2, 8, 2, 64, 64, 16, 8, 1.0, 0, None, 0, 1, None) == -3  # misaligned pool
+    # pool rows num_blocks * K * block_size are TMA row coordinates: below 2^31
+    assert f(P, P, P, P, P, P, 2, 8, 8, 64, 1 << 20, 256, 8, 1.0, 0, None, 0, 1, None) == -2
+    # a split plan needs a workspace
+    assert f(P, P, P, P, P, P, 1, 8, 2, 64, 2048, 16, 2048, 1.0, 0, None, 0, 1, None) == -1
+    assert f(None, None, None, None, None, None, 0, 8, 2, 64, 64, 16, 8, 1.0, 0, None, 0, 1, None) == 0
+    fa = lib.gqa_decode_append_paged
+    assert fa(P, P, P, P, P, P, P, P, 2, 8, 2, 64, 64, 40, 8, 1.0, 0, None, 0, 1, None) == -2
+    assert fa(P, P, P, P, None, P, P, P, 2, 8, 2, 64, 64, 16, 8, 1.0, 0, None, 0, 1, None) == -1  # no k_new
+    ap = lib.gqa_kv_append_paged
+    # k_pool, v_pool, k_new, v_new, table, pos, B, K, d, num_blocks, block_size, max_blocks, dtype, stream
+    assert ap(P, P, P, P, P, P, 2, 2, 64, 64, 8, 8, 1, None) == -2      # block size not 16k
+    assert ap(P, P, P, P, None, P, 2, 2, 64, 64, 16, 8, 1, None) == -1  # no table
+    assert ap(P, P, P, P, P, P, 2, 2, 72, 64, 16, 8, 1, None) == -2     # head dim
+    assert ap(None, None, None, None, None, None, 0, 2, 64, 64, 16, 8, 1, None) == 0
+    ws = lib.gqa_decode_paged_workspace_bytes
+    assert ws(1, 8, 2, 64, 24, 8, 0) == 0 and ws(1, 6, 4, 64, 16, 8, 0) == 0
+    assert ws(1, 64, 8, 128, 16, 8192, 0) > 0  # a long sequence is split
 
 
 def test_prefill_rejects_bad_arguments(lib):
