@@ -82,25 +82,50 @@ __device__ __forceinline__ void wide_tile_blocks(const DecodeParams& p, int b, i
     tr.r16[bx] = bx < tr.n16 ? __ldg(row + (t0 + tr.n64 * kWideBox + bx * kDecBoxRows) / p.block_size) : 0;
 }
 
-template <bool kPaged>
-__device__ __forceinline__ void wide_tile_rows(const DecodeParams& p, int b, int g, int t0, WideTileRows& tr) {
+__device__ __forceinline__ void wide_tile_rows(const DecodeParams& p, int g, int t0, WideTileRows& tr) {
 #pragma unroll
   for (int bx = 0; bx < kWideKeys / kWideBox; ++bx) {
     if (bx >= tr.n64) break;
-    const int t = t0 + bx * kWideBox;
-    tr.r64[bx] = kPaged ? paged_row(p, tr.r64[bx], g, t) : kv_row<false>(p, b, g, t);
+    tr.r64[bx] = paged_row(p, tr.r64[bx], g, t0 + bx * kWideBox);
   }
 #pragma unroll
   for (int bx = 0; bx < kWideKeys / kDecBoxRows; ++bx) {
     if (bx >= tr.n16) break;
-    const int t = t0 + tr.n64 * kWideBox + bx * kDecBoxRows;
-    tr.r16[bx] = kPaged ? paged_row(p, tr.r16[bx], g, t) : kv_row<false>(p, b, g, t);
+    tr.r16[bx] = paged_row(p, tr.r16[bx], g, t0 + tr.n64 * kWideBox + bx * kDecBoxRows);
   }
 }
 
+// The contiguous cache: the tile's rows start at row0.
 __device__ __forceinline__ void wide_issue_tile(uint8_t* stage, uint64_t* full, const CUtensorMap* tm_k64,
                                                 const CUtensorMap* tm_v64, const CUtensorMap* tm_k16,
-                                                const CUtensorMap* tm_v16, const WideTileRows& tr, uint64_t policy) {
+                                                const CUtensorMap* tm_v16, int row0, int rows, uint64_t policy) {
+  using C = WideCfg;
+  const int n64 = rows / kWideBox;
+  const int rem = rows - n64 * kWideBox;
+  const int n16 = (rem + kDecBoxRows - 1) / kDecBoxRows;
+  mbar_arrive_expect_tx(full, (uint32_t)((n64 * kWideBox + n16 * kDecBoxRows) * 128 * 2 * 2));
+  for (int bx = 0; bx < n64; ++bx)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int off = hf * C::kHalf + bx * kWideBox * 128;
+      tma_load_2d(stage + off, tm_k64, hf * 64, row0 + bx * kWideBox, full, policy);
+      tma_load_2d(stage + C::kTile + off, tm_v64, hf * 64, row0 + bx * kWideBox, full, policy);
+    }
+  for (int bx = 0; bx < n16; ++bx)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int r = n64 * kWideBox + bx * kDecBoxRows;
+      const int off = hf * C::kHalf + r * 128;
+      tma_load_2d(stage + off, tm_k16, hf * 64, row0 + r, full, policy);
+      tma_load_2d(stage + C::kTile + off, tm_v16, hf * 64, row0 + r, full, policy);
+    }
+}
+
+// A paged pool: each box at the row wide_tile_rows found for it.
+__device__ __forceinline__ void wide_issue_tile_paged(uint8_t* stage, uint64_t* full, const CUtensorMap* tm_k64,
+                                                      const CUtensorMap* tm_v64, const CUtensorMap* tm_k16,
+                                                      const CUtensorMap* tm_v16, const WideTileRows& tr,
+                                                      uint64_t policy) {
   using C = WideCfg;
   mbar_arrive_expect_tx(full, (uint32_t)((tr.n64 * kWideBox + tr.n16 * kDecBoxRows) * 128 * 2 * 2));
 #pragma unroll
@@ -301,26 +326,36 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         ++nq;
         const int ntiles = (t_end - t_begin + kWideKeys - 1) / kWideKeys;
         WideTileRows tr_next;
-        wide_tile_shape<kPaged>(p, min(kWideKeys, t_end - t_begin), tr_next);
-        if constexpr (kPaged) wide_tile_blocks(p, c.b, t_begin, tr_next);
+        if constexpr (kPaged) {
+          wide_tile_shape<true>(p, min(kWideKeys, t_end - t_begin), tr_next);
+          wide_tile_blocks(p, c.b, t_begin, tr_next);
+        }
         for (int tt = 0; tt < ntiles && ok; ++tt, ++it) {
           const int s = it % C::kStages;
           const int t0 = t_begin + tt * kWideKeys;
           const int rows = min(kWideKeys, t_end - t0);
-          WideTileRows tr = tr_next;
-          if (tt + 1 < ntiles) {  // a paged cache's next table entries load during the wait
-            wide_tile_shape<kPaged>(p, min(kWideKeys, t_end - t0 - kWideKeys), tr_next);
-            if constexpr (kPaged) wide_tile_blocks(p, c.b, t0 + kWideKeys, tr_next);
+          WideTileRows tr;
+          if constexpr (kPaged) {  // this tile's table entries; the next tile's load during the wait
+            tr = tr_next;
+            if (tt + 1 < ntiles) {
+              wide_tile_shape<true>(p, min(kWideKeys, t_end - t0 - kWideKeys), tr_next);
+              wide_tile_blocks(p, c.b, t0 + kWideKeys, tr_next);
+            }
           }
           if (it >= C::kStages) ok = mbar_wait_bounded(&kv_empty[s], ((it / C::kStages) - 1) & 1);
           if (!ok) break;
-          wide_tile_rows<kPaged>(p, c.b, c.g, t0, tr);
           info[s] = StageInfo{item, rows,
                               (tt == 0 ? kTileFirst : 0) | (tt == ntiles - 1 ? kTileLast : 0) |
                                   (len <= p.chunk ? kUnitSingleSplit : 0),
                               -1};
-          wide_issue_tile(smem + C::kKVOff + s * C::kStage, &kv_full[s], &tm_k64, &tm_v64, &tm_k16, &tm_v16, tr,
-                          policy);
+          if constexpr (kPaged) {
+            wide_tile_rows(p, c.g, t0, tr);
+            wide_issue_tile_paged(smem + C::kKVOff + s * C::kStage, &kv_full[s], &tm_k64, &tm_v64, &tm_k16,
+                                  &tm_v16, tr, policy);
+          } else {
+            wide_issue_tile(smem + C::kKVOff + s * C::kStage, &kv_full[s], &tm_k64, &tm_v64, &tm_k16, &tm_v16,
+                            c.unit * p.S_max + t0, rows, policy);
+          }
         }
         if (!ok) break;
       }
