@@ -18,6 +18,15 @@ Page citations (title, section):
   * KV append: "分組查詢注意力", section 技術原理 (each new token writes K and
     V of shape [batch, 1, K, d_k]); "GQA 完全拆解", section 解码推理的内存账本
     (after step t the new K, V row is appended to the cache).
+  * 8-bit KV cache: "GQA 完全拆解", section 更进一步的 KV 压缩 (the cache's K and
+    V held as INT8 instead of FP16, orthogonal to GQA: GQA reduces the head
+    count, quantization the bytes per element) and "LLaMa3与DeepSeek采用的GQA
+    技术", deployment advice (an 8-bit KV cache halves its memory again). The
+    pages give no scale convention; the reading used here: symmetric int8
+    codes in [-127, 127] with one float32 scale per cached row (token and KV
+    head), value = code * scale; quantization in float32: scale = amax / 127,
+    code = round-half-even(x / scale). Decoding an 8-bit cache is the decode
+    of the values it holds.
   * Paged KV cache: "分組查詢注意力", section 下游 / 推論引擎與架構 (the
     paged cache manages blocks of the K KV heads, not of the H query heads,
     and each block is broadcast to the group's H/K query heads when it is
@@ -85,6 +94,10 @@ def _declare(lib):
     lib.ref_prefill_causal.argtypes = [P, P, P, P, I, I, I, I, I, D, I, P, I64, I]
     lib.ref_meanpool.restype = I
     lib.ref_meanpool.argtypes = [P, P, I64, I, I, I64, I]
+    lib.ref_decode_int8.restype = I
+    lib.ref_decode_int8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, D, I, P, I64, I]
+    lib.ref_quantize_int8.restype = None
+    lib.ref_quantize_int8.argtypes = [P, P, P, I, I64, I]
     lib.ref_round_bf16.argtypes = [P, P, I64]
     lib.ref_round_f32.argtypes = [P, P, I64]
     return lib
@@ -298,3 +311,65 @@ def kv_append_paged(k_pool, v_pool, k_new, v_new, block_table, pos):
             kp[blk, :, p % bs, :] = k_new[b]
             vp[blk, :, p % bs, :] = v_new[b]
     return kp, vp
+
+
+# ---------------------------------------------------------------------------
+# 8-bit KV cache: codes int8 [..., d], one float32 scale per row
+
+def quantize_int8(x, lib=None):
+    """x [..., n] (float64, float32 or bfloat16 bits) -> (codes int8 [..., n], scales float32 [...])."""
+    x = _c(x)
+    n = x.shape[-1]
+    rows = x.size // n if n else 0
+    codes = np.empty(x.shape, dtype=np.int8)
+    scales = np.empty(x.shape[:-1], dtype=np.float32)
+    if rows:
+        _get(lib).ref_quantize_int8(codes.ctypes.data, scales.ctypes.data, x.ctypes.data, _dtype_code(x), rows, n)
+    return codes, scales
+
+
+def dequantize_int8(codes, scales) -> np.ndarray:
+    """code * scale in float64 (exact)."""
+    return codes.astype(np.float64) * scales.astype(np.float64)[..., None]
+
+
+def decode_int8(q, k_codes, k_scales, v_codes, v_scales, seqlens, scale: float, sel=None, nthreads=None,
+                lib=None) -> np.ndarray:
+    """q [B,H,d]; k/v codes [B,K,S_max,d] int8, scales [B,K,S_max] float32 -> float64 [B,H,d] (or [len(sel), d])."""
+    q = _c(q)
+    k_codes, v_codes = _c(k_codes).astype(np.int8, copy=False), _c(v_codes).astype(np.int8, copy=False)
+    k_scales = np.ascontiguousarray(k_scales, dtype=np.float32)
+    v_scales = np.ascontiguousarray(v_scales, dtype=np.float32)
+    B, H, d = q.shape
+    Bk, K, S_max, dk = k_codes.shape
+    assert Bk == B and dk == d and v_codes.shape == k_codes.shape
+    assert k_scales.shape == (B, K, S_max) and v_scales.shape == k_scales.shape
+    seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
+    if sel is None:
+        out = np.empty((B, H, d), dtype=np.float64)
+        selp, nsel = None, 0
+    else:
+        sel = np.ascontiguousarray(sel, dtype=np.int32).reshape(-1, 2)
+        out = np.empty((sel.shape[0], d), dtype=np.float64)
+        selp, nsel = sel.ctypes.data, sel.shape[0]
+    rc = _get(lib).ref_decode_int8(out.ctypes.data, q.ctypes.data, k_codes.ctypes.data, k_scales.ctypes.data,
+                                   v_codes.ctypes.data, v_scales.ctypes.data, seqlens.ctypes.data, B, H, K, S_max, d,
+                                   float(scale), _dtype_code(q), selp, nsel, _threads(nthreads))
+    if rc != 0:
+        raise ValueError("oracle: H must be a multiple of K")
+    return out
+
+
+def kv_append_int8(k_codes, k_scales, v_codes, v_scales, k_new, v_new, pos, lib=None):
+    """Copies of the 8-bit caches with key pos[b] of every (b, g) set to the quantized new token
+    (k_new/v_new [B,K,d]); positions outside [0, S_max) leave the caches untouched."""
+    kc, ks, vc, vs = (np.array(a, copy=True) for a in (k_codes, k_scales, v_codes, v_scales))
+    B, K, S_max, _ = kc.shape
+    kq, kqs = quantize_int8(k_new, lib)
+    vq, vqs = quantize_int8(v_new, lib)
+    for b in range(B):
+        p = int(pos[b])
+        if 0 <= p < S_max:
+            kc[b, :, p], ks[b, :, p] = kq[b], kqs[b]
+            vc[b, :, p], vs[b, :, p] = vq[b], vqs[b]
+    return kc, ks, vc, vs

@@ -44,6 +44,7 @@
 #define REF_F32 0
 #define REF_BF16 1
 #define REF_F64 2
+#define REF_I8 3 /* caches only: int8 codes, one float scale per row of d */
 
 /* exact widening of one stored element to double */
 static double widen(const void* base, int dtype, int64_t i) {
@@ -87,13 +88,26 @@ void ref_round_f32(const double* x, float* out, int64_t n) {
   for (int64_t i = 0; i < n; ++i) out[i] = (float)x[i];
 }
 
+/* A K or V cache as stored: elements of `dtype`, or int8 codes whose value
+ * is code * scales[row] (row = element index / d), exact in double. */
+typedef struct {
+  const void* base;
+  const float* scales;
+  int dtype;
+  int d;
+} kv_src;
+
+static double widen_kv(const kv_src* c, int64_t i) {
+  if (c->dtype == REF_I8) return (double)((const int8_t*)c->base)[i] * (double)c->scales[i / c->d];
+  return widen(c->base, c->dtype, i);
+}
+
 /* ------------------------------------------------------------------------ */
 /* attention of one query row against keys 0..n-1 of one KV head            */
 
-/* q: d values at q_base+q_off; key t: k_base + k_off + t*k_stride (d values) */
-static void attend_row(double* out, const void* q, int64_t q_off, const void* k, const void* v,
-                       int64_t kv_off, int64_t kv_stride, int64_t n, int d, double scale, int dtype,
-                       double* s) {
+/* q: d values at q + q_off; key t: element kv_off + t*kv_stride of k (d values) */
+static void attend_row(double* out, const void* q, int64_t q_off, int q_dtype, const kv_src* k, const kv_src* v,
+                       int64_t kv_off, int64_t kv_stride, int64_t n, int d, double scale, double* s) {
   if (n <= 0) {
     for (int i = 0; i < d; ++i) out[i] = 0.0;
     return;
@@ -101,7 +115,7 @@ static void attend_row(double* out, const void* q, int64_t q_off, const void* k,
   /* scores s_t = scale * sum_i q_i k_{t,i} */
   for (int64_t t = 0; t < n; ++t) {
     double acc = 0.0;
-    for (int i = 0; i < d; ++i) acc += widen(q, dtype, q_off + i) * widen(k, dtype, kv_off + t * kv_stride + i);
+    for (int i = 0; i < d; ++i) acc += widen(q, q_dtype, q_off + i) * widen_kv(k, kv_off + t * kv_stride + i);
     s[t] = scale * acc;
   }
   /* two-pass softmax: m = max_t s_t, w_t = exp(s_t - m), Z = sum_t w_t */
@@ -117,7 +131,7 @@ static void attend_row(double* out, const void* q, int64_t q_off, const void* k,
   for (int i = 0; i < d; ++i) out[i] = 0.0;
   for (int64_t t = 0; t < n; ++t) {
     double w = s[t];
-    for (int i = 0; i < d; ++i) out[i] += w * widen(v, dtype, kv_off + t * kv_stride + i);
+    for (int i = 0; i < d; ++i) out[i] += w * widen_kv(v, kv_off + t * kv_stride + i);
   }
   for (int i = 0; i < d; ++i) out[i] /= Z;
 }
@@ -127,11 +141,12 @@ static void attend_row(double* out, const void* q, int64_t q_off, const void* k,
 
 typedef struct {
   double* out;
-  const void *q, *kc, *vc;
+  const void* q;
+  kv_src kc, vc;
   const int32_t* seqlens;
   int B, H, K, S_max, d;
   double scale;
-  int dtype;
+  int dtype; /* of q */
   const int32_t* sel; /* nsel (b, h) pairs, or NULL for every (b, g) unit */
   int64_t nsel;
   int64_t next;       /* work counter, protected by mu */
@@ -153,7 +168,7 @@ static void decode_head(decode_job* jb, int b, int h, double* dst, double* s) {
   if (n > jb->S_max) n = jb->S_max;
   int64_t q_off = ((int64_t)b * jb->H + h) * jb->d;
   int64_t kv_off = ((int64_t)b * jb->K + g) * jb->S_max * jb->d;
-  attend_row(dst, jb->q, q_off, jb->kc, jb->vc, kv_off, jb->d, n, jb->d, jb->scale, jb->dtype, s);
+  attend_row(dst, jb->q, q_off, jb->dtype, &jb->kc, &jb->vc, kv_off, jb->d, n, jb->d, jb->scale, s);
 }
 
 static void* decode_worker(void* arg) {
@@ -198,11 +213,58 @@ int ref_decode(double* out, const void* q, const void* k_cache, const void* v_ca
                int B, int H, int K, int S_max, int d, double scale, int dtype, const int32_t* sel,
                int64_t nsel, int nthreads) {
   if (K <= 0 || H <= 0 || H % K != 0 || d <= 0 || B < 0 || S_max < 0) return -1;
-  decode_job jb = {out, q, k_cache, v_cache, seqlens, B, H, K, S_max, d, scale, dtype, sel, nsel, 0};
+  decode_job jb = {out, q, {k_cache, NULL, dtype, d}, {v_cache, NULL, dtype, d}, seqlens, B, H, K, S_max, d,
+                   scale, dtype, sel, nsel, 0};
   pthread_mutex_init(&jb.mu, NULL);
   run_threads(decode_worker, &jb, nthreads);
   pthread_mutex_destroy(&jb.mu);
   return 0;
+}
+
+/* The same over an 8-bit cache: k_codes/v_codes [B,K,S_max,d] int8 with one
+ * float scale per row (k_scales/v_scales [B,K,S_max]); the cached value is
+ * code * scale ("GQA 完全拆解", section 更进一步的 KV 压缩: the cache's K and V
+ * held as INT8). q has q_dtype. */
+int ref_decode_int8(double* out, const void* q, const int8_t* k_codes, const float* k_scales, const int8_t* v_codes,
+                    const float* v_scales, const int32_t* seqlens, int B, int H, int K, int S_max, int d,
+                    double scale, int q_dtype, const int32_t* sel, int64_t nsel, int nthreads) {
+  if (K <= 0 || H <= 0 || H % K != 0 || d <= 0 || B < 0 || S_max < 0) return -1;
+  decode_job jb = {out, q, {k_codes, k_scales, REF_I8, d}, {v_codes, v_scales, REF_I8, d}, seqlens, B, H, K, S_max,
+                   d, scale, q_dtype, sel, nsel, 0};
+  pthread_mutex_init(&jb.mu, NULL);
+  run_threads(decode_worker, &jb, nthreads);
+  pthread_mutex_destroy(&jb.mu);
+  return 0;
+}
+
+/* Symmetric 8-bit quantization of `rows` rows of n elements (x of dtype
+ * REF_BF16, REF_F32 or REF_F64 read as float), in float arithmetic as
+ * written: amax = max_i |x_i|; scale = amax / 127; code_i = x_i / scale
+ * rounded to nearest, ties to even, clamped to [-127, 127]; a row of zeros
+ * gets scale 0 and codes 0. The pages name 8-bit KV caches ("GQA 完全拆解",
+ * section 更进一步的 KV 压缩; "LLaMa3与DeepSeek采用的GQA技术", deployment
+ * advice) without a scale convention; this per-row symmetric one is the
+ * reading taken. Float, not double: a code is an integer decided by floating
+ * point, and both implementations decide it in the same precision. */
+void ref_quantize_int8(int8_t* codes, float* scales, const void* x, int dtype, int64_t rows, int n) {
+  for (int64_t r = 0; r < rows; ++r) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+      float a = fabsf((float)widen(x, dtype, r * n + i));
+      if (a > amax) amax = a;
+    }
+    float sc = amax / 127.0f;
+    scales[r] = sc;
+    for (int i = 0; i < n; ++i) {
+      float c = 0.0f;
+      if (sc > 0.0f) {
+        c = nearbyintf((float)widen(x, dtype, r * n + i) / sc); /* default rounding: nearest, ties to even */
+        if (c > 127.0f) c = 127.0f;
+        if (c < -127.0f) c = -127.0f;
+      }
+      codes[r * n + i] = (int8_t)c;
+    }
+  }
 }
 
 /* ------------------------------------------------------------------------ */
@@ -211,7 +273,8 @@ int ref_decode(double* out, const void* q, const void* k_cache, const void* v_ca
 
 typedef struct {
   double* out;
-  const void *q, *k, *v;
+  const void* q;
+  kv_src k, v;
   int B, S, H, K, d;
   double scale;
   int dtype;
@@ -226,8 +289,8 @@ static void prefill_row(prefill_job* jb, int b, int i, int h, double* dst, doubl
   int g = h / G;
   int64_t q_off = (((int64_t)b * jb->S + i) * jb->H + h) * jb->d;
   int64_t kv_off = ((int64_t)b * jb->S * jb->K + g) * jb->d; /* key j at kv_off + j*K*d */
-  attend_row(dst, jb->q, q_off, jb->k, jb->v, kv_off, (int64_t)jb->K * jb->d, (int64_t)i + 1, jb->d,
-             jb->scale, jb->dtype, s);
+  attend_row(dst, jb->q, q_off, jb->dtype, &jb->k, &jb->v, kv_off, (int64_t)jb->K * jb->d, (int64_t)i + 1, jb->d,
+             jb->scale, s);
 }
 
 static void* prefill_worker(void* arg) {
@@ -259,7 +322,7 @@ static void* prefill_worker(void* arg) {
 int ref_prefill_causal(double* out, const void* q, const void* k, const void* v, int B, int S, int H, int K,
                        int d, double scale, int dtype, const int32_t* sel, int64_t nsel, int nthreads) {
   if (K <= 0 || H <= 0 || H % K != 0 || d <= 0 || B < 0 || S < 0) return -1;
-  prefill_job jb = {out, q, k, v, B, S, H, K, d, scale, dtype, sel, nsel, 0};
+  prefill_job jb = {out, q, {k, NULL, dtype, d}, {v, NULL, dtype, d}, B, S, H, K, d, scale, dtype, sel, nsel, 0};
   pthread_mutex_init(&jb.mu, NULL);
   run_threads(prefill_worker, &jb, nthreads);
   pthread_mutex_destroy(&jb.mu);

@@ -28,6 +28,7 @@ _LIB = os.path.join(_HERE, "libsynth.so")
 F32, BF16, F64 = 0, 1, 2
 SEED_BASE = 0x6A510000
 STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_KNEW, STREAM_VNEW, STREAM_BLOCKS = 1, 2, 3, 4, 5, 6, 7
+STREAM_K8, STREAM_V8, STREAM_KSCALE, STREAM_VSCALE = 10, 11, 12, 13
 
 
 def build(force: bool = False) -> str:
@@ -56,6 +57,9 @@ def _get():
                                     ctypes.c_int]
         lib.synth_uniform_int.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int64,
                                           ctypes.c_int32, ctypes.c_int32]
+        lib.synth_int8_cache.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint64,
+                                         ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                         ctypes.c_int64, ctypes.c_float, ctypes.c_float]
         _lib = lib
     return _lib
 
@@ -270,3 +274,43 @@ def paged_inputs(pw: PagedShape) -> dict:
     inp.update(page(inp["k_cache"], inp["v_cache"], lens, pw.block_size, pw.spare_blocks, w.seed,
                     append_row=w.append))
     return inp
+
+
+# --------------------------------------------------------------------------
+# 8-bit caches: random codes and per-row scales (no quantizer here: the codes
+# are data, the scales are in the range a row of N(0, 1) values would get)
+
+
+def int8_cache(units: int, S_max: int, d: int, seed: int, stream_codes: int, stream_scales: int,
+               lens: Optional[np.ndarray] = None, units_per_len: int = 1, lo: float = 0.015, hi: float = 0.035):
+    """(codes int8 [units, S_max, d] uniform over [-127, 127], scales float32 [units, S_max] uniform
+    over [lo, hi)); rows at or past lens[u // units_per_len] hold code -128 and a NaN scale."""
+    codes = np.empty((units, S_max, d), dtype=np.int8)
+    scales = np.empty((units, S_max), dtype=np.float32)
+    lp = None
+    if lens is not None:
+        lens = np.ascontiguousarray(lens, dtype=np.int32)
+        lp = lens.ctypes.data
+    if codes.size:
+        _get().synth_int8_cache(codes.ctypes.data, scales.ctypes.data, stream_key(seed, stream_codes),
+                                stream_key(seed, stream_scales), units, S_max, d, lp, units_per_len, lo, hi)
+    return codes, scales
+
+
+INT8_WORKLOADS = {
+    "int8_llama3_8b_decode_b8_h32_k8_d128_s8192": "llama3_8b_decode_b8_h32_k8_d128_s8192",
+    "int8_ragged_70b_decode_b32_h64_k8_d128_s1k_16k": "ragged_70b_decode_b32_h64_k8_d128_s1k_16k",
+}
+
+
+def int8_inputs(name: str) -> dict:
+    """q [B,H,d] (the base workload's), 8-bit caches of the base workload's shape and lengths:
+    k_codes/v_codes [B,K,S_max,d] int8, k_scale/v_scale [B,K,S_max] float32, seqlens [B]."""
+    w = DECODE_WORKLOADS[INT8_WORKLOADS[name]]
+    lens = seqlens_for(w)
+    kc, ks = int8_cache(w.B * w.K, w.S_max, w.d, w.seed, STREAM_K8, STREAM_KSCALE, lens, w.K)
+    vc, vs = int8_cache(w.B * w.K, w.S_max, w.d, w.seed, STREAM_V8, STREAM_VSCALE, lens, w.K)
+    shp = (w.B, w.K, w.S_max)
+    return {"q": normal((w.B, w.H, w.d), BF16, w.seed, STREAM_Q), "k_codes": kc.reshape(*shp, w.d),
+            "k_scale": ks.reshape(shp), "v_codes": vc.reshape(*shp, w.d), "v_scale": vs.reshape(shp),
+            "seqlens": lens}

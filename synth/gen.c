@@ -190,3 +190,26 @@ void synth_uniform_int(int32_t* out, uint64_t key, int64_t n, int32_t lo, int32_
   uint64_t span = (uint64_t)((int64_t)hi - (int64_t)lo + 1);
   for (int64_t i = 0; i < n; ++i) out[i] = (int32_t)((int64_t)lo + (int64_t)(draw(key, (uint64_t)i) % span));
 }
+
+/* 8-bit cache rows: codes uniform over [-127, 127] (one draw each, element
+ * (u, t, c) at index (u * S_max + t) * d + c), one scale per row uniform
+ * over [lo, hi) (row index u * S_max + t of a second stream); rows at or past
+ * lens[u / units_per_len] get code -128 and a quiet-NaN scale. */
+void synth_int8_cache(int8_t* codes, float* scales, uint64_t key_codes, uint64_t key_scales, int64_t units,
+                      int64_t S_max, int64_t d, const int32_t* lens, int64_t units_per_len, float lo, float hi) {
+  const float qnan = __builtin_nanf("");
+  for (int64_t u = 0; u < units; ++u) {
+    const int64_t n = lens ? (int64_t)lens[u / units_per_len] : S_max;
+    for (int64_t t = 0; t < S_max; ++t) {
+      const uint64_t row = (uint64_t)(u * S_max + t);
+      int8_t* dst = codes + row * (uint64_t)d;
+      if (t >= n) {
+        for (int64_t c = 0; c < d; ++c) dst[c] = (int8_t)-128;
+        scales[row] = qnan;
+        continue;
+      }
+      for (int64_t c = 0; c < d; ++c) dst[c] = (int8_t)((int)(draw(key_codes, row * (uint64_t)d + c) % 255u) - 127);
+      scales[row] = lo + (hi - lo) * (float)((double)(draw(key_scales, row) >> 11) * 0x1.0p-53);
+    }
+  }
+}

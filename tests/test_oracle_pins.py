@@ -316,7 +316,7 @@ MUTANTS = {
     "round_robin_heads": ("int g = h / G; /* contiguous grouping", "int g = h % jb->K; /* contiguous grouping"),
     "dropped_scale": ("s[t] = scale * acc;", "s[t] = acc;"),
     "unnormalised": ("out[i] /= Z;", "out[i] /= 1.0;"),
-    "k_for_v": ("out[i] += w * widen(v, dtype,", "out[i] += w * widen(k, dtype,"),
+    "k_for_v": ("out[i] += w * widen_kv(v, kv_off", "out[i] += w * widen_kv(k, kv_off"),
     "no_max_subtraction": ("s[t] = exp(s[t] - m);", "s[t] = exp(s[t]);"),
     "ignores_seqlens": ("int64_t n = jb->seqlens[b];", "int64_t n = jb->S_max;"),
     "causal_excludes_diagonal": ("(int64_t)i + 1, jb->d,", "(int64_t)i, jb->d,"),

@@ -82,3 +82,16 @@ def test_paged_inputs_map_the_append_row():
     kc = np.zeros((w.B, 1, w.S_max, 2), dtype=np.uint16)  # a tiny stand-in cache with the same lengths
     pg = synth.page(kc, kc, pos, 16, 2, w.seed, append_row=True)
     assert (pg["block_table"][np.arange(w.B), pos // 16] >= 0).all()
+
+
+def test_int8_cache_codes_scales_and_padding():
+    lens = np.array([5, 0], np.int32)
+    c, s = synth.int8_cache(4, 8, 16, 77, synth.STREAM_K8, synth.STREAM_KSCALE, lens, 2, lo=0.01, hi=0.02)
+    assert c.dtype == np.int8 and s.dtype == np.float32 and c.shape == (4, 8, 16) and s.shape == (4, 8)
+    valid = np.zeros((4, 8), bool)
+    valid[:2, :5] = True
+    assert (c[valid] >= -127).all() and (c[valid] <= 127).all() and len(np.unique(c[valid])) > 50
+    assert (s[valid] >= 0.01).all() and (s[valid] < 0.02).all()
+    assert (c[~valid] == -128).all() and np.isnan(s[~valid]).all()
+    c2, s2 = synth.int8_cache(4, 8, 16, 77, synth.STREAM_K8, synth.STREAM_KSCALE, lens, 2, lo=0.01, hi=0.02)
+    assert np.array_equal(c, c2) and np.array_equal(s[valid], s2[valid])
