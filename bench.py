@@ -291,6 +291,7 @@ DECODE_EXTRA = ["ragged_70b_decode_b32_h64_k8_d128_s1k_16k", "long_ctx_gqa_b1_h6
                 "long_ctx_mqa_b1_h64_k1_d128_s131072"]
 PREFILL = "causal_prefill_b4_s4096_h32_k8_d128"
 PAGED_EXTRA = list(synth.PAGED_WORKLOADS)
+INT8_EXTRA = list(synth.INT8_WORKLOADS)
 
 
 class L2Flush:
@@ -354,6 +355,10 @@ def extra_measurements(args, only=None):
         if only is not None and name != only:
             continue
         res[name] = paged_measurement(args, name, peaks, 20 if only is None else args.steps)
+    for name in INT8_EXTRA:
+        if only is not None and name != only:
+            continue
+        res[name] = int8_measurement(args, name, peaks, 20 if only is None else args.steps)
     if only is not None and only != PREFILL:
         return res
     # causal prefill with the KV-cache write: FLOPs over the causal pairs (j <= i) only
@@ -444,6 +449,49 @@ def paged_measurement(args, name, peaks, steps):
     return r
 
 
+def int8_measurement(args, name, peaks, steps):
+    """gqa_decode_int8 over an 8-bit cache: bytes = the codes and scales of every valid row."""
+    import torch
+
+    from kv_cache_02_b200 import gqa
+
+    inp = synth.int8_inputs(name)
+    B, H, d = inp["q"].shape
+    K, S_max = inp["k_codes"].shape[1:3]
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).cuda()
+
+    q, kc, ks, vc, vs = (to_dev(inp[k]) for k in ("q", "k_codes", "k_scale", "v_codes", "v_scale"))
+    sl = to_dev(inp["seqlens"])
+    out = torch.empty_like(q)
+    wsb = gqa.gqa_decode_int8_workspace_bytes(B, H, K, S_max, d, 0)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+    kv_bytes = int(inp["seqlens"].astype(np.int64).sum()) * K * (d + 4) * 2
+    flush = L2Flush()
+    times = []
+    for it in range(args.warmup + steps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        gqa.gqa_decode_int8(out, q, kc, ks, vc, vs, sl, 1.0 / np.sqrt(d), 0, ws)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            times.append(a.elapsed_time(b))
+    if gqa.gqa_get_last_error() != (0, 0):
+        raise RuntimeError(f"device error in {name}")
+    ms = statistics.median(times)
+    gbs = kv_bytes / (ms * 1e-3) / 1e9
+    r = {"ms": round(ms, 5), "kv_bytes": kv_bytes, "GB/s": round(gbs, 1),
+         "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "call": "gqa_decode_int8",
+         "bytes": "int8 codes + one float scale per row", "l2": "flushed (512 MiB write, then 512 MiB read)"}
+    del q, kc, ks, vc, vs, out, ws, flush
+    torch.cuda.empty_cache()
+    return r
+
+
 def cpu_baseline(inp, scale, kv_bytes_layer):
     """The oracle as it stands, on all host cores, over one full layer of the workload."""
     import oracle
@@ -498,7 +546,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads and the CPU baseline")
-    ap.add_argument("--only", choices=DECODE_EXTRA + PAGED_EXTRA + [PREFILL], default=None,
+    ap.add_argument("--only", choices=DECODE_EXTRA + PAGED_EXTRA + INT8_EXTRA + [PREFILL], default=None,
                     help="time one other workload alone (for profiling); prints its own JSON, not the contract line")
     ap.add_argument("--layers", type=int, default=32,
                     help="layers per step (32 for the model; fewer only for small profiling captures)")

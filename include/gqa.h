@@ -230,6 +230,42 @@ GQA_API int gqa_kv_append_paged(void* k_pool, void* v_pool, const void* k_new, c
                                 int block_size, int max_blocks, gqa_dtype dtype, gqa_stream_t stream);
 
 /*
+ * 8-bit KV cache: gqa_kv_append_int8 and gqa_decode_int8.
+ *
+ * "GQA 完全拆解", section 更进一步的 KV 压缩: the cache's K and V held as INT8
+ * instead of FP16, orthogonal to GQA (GQA reduces the head count,
+ * quantization the bytes per element); "LLaMa3与DeepSeek采用的GQA技术",
+ * deployment advice: an 8-bit KV cache halves its memory again. The pages
+ * give no scale convention; here:
+ *
+ *   value[b, g, t, i] = k_codes[b, g, t, i] * k_scales[b, g, t]   (V likewise)
+ *
+ * k_codes, v_codes   : [B, K, S_max, d] int8, codes in [-127, 127].
+ * k_scales, v_scales : [B, K, S_max] float32, one scale per cached row.
+ * d must be 128 and S_max a multiple of 4 (GQA_ERR_UNSUPPORTED /
+ * GQA_ERR_SHAPE otherwise).
+ *
+ * gqa_kv_append_int8 quantizes the new token's rows k_new, v_new ([B, K, d]
+ * bfloat16) into key pos[b]: scale = amax / 127 and code = x / scale rounded
+ * to nearest (ties to even) and clamped to [-127, 127], in float with
+ * correctly rounded divisions (a row of zeros: scale 0, codes 0). pos as for
+ * gqa_kv_append (GQA_DEVERR_APPEND_POS outside [0, S_max)).
+ *
+ * gqa_decode_int8 is gqa_decode over the values the 8-bit cache holds: q and
+ * out are [B, H, d] bfloat16, everything else (seqlens, scale, num_splits,
+ * the workspace of gqa_decode_int8_workspace_bytes bytes, errors) as for
+ * gqa_decode. Rows t >= len_b are never read into the result.
+ */
+GQA_API size_t gqa_decode_int8_workspace_bytes(int B, int H, int K, int S_max, int d, int num_splits);
+GQA_API int gqa_decode_int8(void* out, const void* q, const int8_t* k_codes, const float* k_scales,
+                            const int8_t* v_codes, const float* v_scales, const int32_t* seqlens, int B, int H,
+                            int K, int S_max, int d, float scale, int num_splits, void* workspace,
+                            size_t workspace_bytes, gqa_stream_t stream);
+GQA_API int gqa_kv_append_int8(int8_t* k_codes, float* k_scales, int8_t* v_codes, float* v_scales,
+                               const void* k_new, const void* v_new, const int32_t* pos, int B, int K, int S_max,
+                               int d, gqa_stream_t stream);
+
+/*
  * gqa_prefill_causal - causal self-attention over a whole prompt, and the
  * write of its keys and values into the cache.
  *

@@ -50,6 +50,48 @@ __global__ void kv_append_kernel(uint4* __restrict__ k_cache, uint4* __restrict_
   }
 }
 
+// gqa_kv_append_int8: the new token's K and V rows (bf16, d = 128) quantized
+// into the 8-bit cache at key pos[b]: scale = amax / 127, code = x / scale
+// rounded to nearest even, clamped to [-127, 127] (a zero row: scale 0,
+// codes 0), in float with correctly rounded divisions. One warp per row
+// (4 values per lane), K rows then V rows.
+__global__ void kv_append_int8_kernel(int8_t* __restrict__ k_codes, float* __restrict__ k_scales,
+                                      int8_t* __restrict__ v_codes, float* __restrict__ v_scales,
+                                      const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __restrict__ v_new,
+                                      const int32_t* __restrict__ pos, int B, int K, int S_max) {
+  constexpr int D = 128;
+  const int lane = threadIdx.x & 31;
+  const long long nrows = (long long)B * K;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); r < 2 * nrows; r += warps) {
+    const bool is_v = r >= nrows;
+    const long long row = is_v ? r - nrows : r;  // b * K + g
+    const int b = (int)(row / K);
+    const int p = __ldg(pos + b);
+    if (p < 0 || p >= S_max) {
+      if (lane == 0 && !is_v && row % K == 0) raise_error(GQA_DEVERR_APPEND_POS);
+      continue;
+    }
+    const uint2 w = __ldg(reinterpret_cast<const uint2*>((is_v ? v_new : k_new) + row * D) + lane);
+    const float x[4] = {__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u), __uint_as_float(w.y << 16),
+                        __uint_as_float(w.y & 0xffff0000u)};
+    float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float sc = __fdiv_rn(amax, 127.0f);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int c = 0;
+      if (sc > 0.f) c = min(127, max(-127, __float2int_rn(__fdiv_rn(x[i], sc))));
+      packed |= (uint32_t)(uint8_t)(int8_t)c << (8 * i);
+    }
+    const long long dst = row * S_max + p;
+    reinterpret_cast<uint32_t*>((is_v ? v_codes : k_codes) + dst * D)[lane] = packed;
+    if (lane == 0) (is_v ? v_scales : k_scales)[dst] = sc;
+  }
+}
+
 // Prompt write: k [B, S, K, d] -> k_cache [B, K, S_max, d] rows 0..S-1 (and V).
 __global__ void kv_write_prompt_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                                        const uint4* __restrict__ k, const uint4* __restrict__ v, int B, int S,

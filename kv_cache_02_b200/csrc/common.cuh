@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -149,6 +150,35 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D(16x8) += A(16x16, row) * B(16x8, col), fp16 operands, fp32 accumulate
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two floats -> packed f16x2 (lo in the low half), round to nearest-even.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Four int8 codes (one 32-bit word, code i in byte i) -> two f16x2 holding
+// them exactly: lo = (code 0, code 1), hi = (code 2, code 3). Biased by 128 a
+// code is a byte u; the f16 with bits 0x64uu is 1024 + u (the 10-bit mantissa
+// holds u exactly), and subtracting 1152 (bits 0x6480) leaves the code.
+__device__ __forceinline__ void int8x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const uint32_t blo = __byte_perm(u, 0x64646464u, 0x5140);  // bytes u0, 0x64, u1, 0x64
+  const uint32_t bhi = __byte_perm(u, 0x64646464u, 0x5342);  // bytes u2, 0x64, u3, 0x64
+  const uint32_t bias = 0x64806480u;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(blo), "r"(bias));
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(bhi), "r"(bias));
 }
 
 // Transpose an 8x8 matrix of 16-bit values held as one m8n8 fragment per warp.

@@ -40,13 +40,21 @@ constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
 constexpr int kDecBoxRows = 16;  // TMA box height; the ragged tail is read in 16-row steps
 constexpr int kDecHeadsPerCta = 8;
 
-template <int D>
+// Ring stage geometry. bf16 cache: K tile then V tile, each in 128-byte
+// column boxes. 8-bit cache (kInt8, d = 128): a key row of codes is one
+// 128-byte swizzled row; K codes, V codes, then the tile's 64 K scales and
+// 64 V scales (float), the stage rounded up to 1024 bytes.
+template <int D, bool kInt8 = false>
 struct DecCfg {
-  static constexpr int kHalves = D / 64;                       // 128-byte column boxes per row
+  static_assert(!kInt8 || D == 128, "the 8-bit cache is laid out for head dim 128");
+  static constexpr int kElt = kInt8 ? 1 : 2;
+  static constexpr int kHalves = D * kElt / 128;               // 128-byte column boxes per row
   static constexpr int kHalfBytes = kDecTileKeys * 128;        // one column box of a tile
-  static constexpr int kTileBytes = kDecTileKeys * D * 2;      // K (or V) tile
-  static constexpr int kStages = (D == 128) ? 3 : 6;
-  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kTileBytes = kDecTileKeys * D * kElt;   // K (or V) tile
+  static constexpr int kScaleOff = 2 * kTileBytes;             // 8-bit: K scales, then V scales
+  static constexpr int kStages = kInt8 ? 5 : ((D == 128) ? 3 : 6);
+  static constexpr int kStageBytes = kInt8 ? (2 * kTileBytes + 2 * kDecTileKeys * 4 + 1023) / 1024 * 1024
+                                           : 2 * kTileBytes;
   static constexpr int kRingBytes = kStages * kStageBytes;
   // merge scratch: per consumer warp, m and l of 8 heads, then O of 8 heads
   static constexpr int kMergeFloats = kDecConsumerWarps * (2 * kDecHeadsPerCta + kDecHeadsPerCta * D);
@@ -226,6 +234,35 @@ __device__ __forceinline__ void issue_tile_paged(uint8_t* stage, uint64_t* full,
   }
 }
 
+// The 8-bit cache: the codes of a full tile as one 64-row box each for K and
+// V, a partial tile as 16-row boxes; the tile's 64 K and 64 V scales as one
+// box each from the [units, S_max] scale arrays (a box reaching past a row's
+// end reads the next unit's scales, past the array's end TMA fills zeros;
+// only scales of valid keys are used).
+template <int D>
+__device__ __forceinline__ void issue_tile_i8(uint8_t* stage, uint64_t* full, const CUtensorMap* tm_k64,
+                                              const CUtensorMap* tm_v64, const CUtensorMap* tm_k16,
+                                              const CUtensorMap* tm_v16, const CUtensorMap* tm_ks,
+                                              const CUtensorMap* tm_vs, int row0, int unit, int t0, int rows,
+                                              uint64_t policy) {
+  using C = DecCfg<D, true>;
+  constexpr uint32_t kScaleBytes = kDecTileKeys * 4;
+  if (rows == kDecTileKeys) {
+    mbar_arrive_expect_tx(full, (uint32_t)(2 * C::kTileBytes) + 2 * kScaleBytes);
+    tma_load_2d(stage, tm_k64, 0, row0, full, policy);
+    tma_load_2d(stage + C::kTileBytes, tm_v64, 0, row0, full, policy);
+  } else {
+    const int nbox = (rows + kDecBoxRows - 1) / kDecBoxRows;
+    mbar_arrive_expect_tx(full, (uint32_t)(nbox * kDecBoxRows * 128 * 2) + 2 * kScaleBytes);
+    for (int bx = 0; bx < nbox; ++bx) {
+      tma_load_2d(stage + bx * kDecBoxRows * 128, tm_k16, 0, row0 + bx * kDecBoxRows, full, policy);
+      tma_load_2d(stage + C::kTileBytes + bx * kDecBoxRows * 128, tm_v16, 0, row0 + bx * kDecBoxRows, full, policy);
+    }
+  }
+  tma_load_2d(stage + C::kScaleOff, tm_ks, t0, unit, full, policy);
+  tma_load_2d(stage + C::kScaleOff + kScaleBytes, tm_vs, t0, unit, full, policy);
+}
+
 // Table entries of the 16-row boxes of the tile of keys t0 .. t0 + rows - 1
 // of sequence b (every block size is a multiple of 16, so a box never
 // straddles blocks): independent loads, consumed only when the tile is
@@ -240,6 +277,25 @@ __device__ __forceinline__ void tile_blocks(const DecodeParams& p, int b, int t0
 
 // Q^T as the B operand (k = dims, n = heads): lane holds head lane/4, dims
 // 2*(lane%4) + {0,1} (b0) and + 8 (b1) of every 16-dim step.
+// Q^T as the fp16 B operand of the 8-bit path: in the 16-dim step ks the
+// lane holds head lane/4, dims 16 ks + 4 (lane%4) + {0, 1} (b0) and
+// + {2, 3} (b1) -- the order in which a key row's codes reach the A operand
+// (warp_tile_i8), so the dot products are unchanged.
+template <int D>
+__device__ __forceinline__ void load_q_frag_i8(uint32_t (&qf)[D / 16][2], const __nv_bfloat16* q, int lane, int nh) {
+  const int hn = lane >> 2;
+  const bool hv = hn < nh;
+  const uint2* qrow = reinterpret_cast<const uint2*>(q + (size_t)(hv ? hn : 0) * D);
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const uint2 w = __ldg(qrow + ks * 4 + (lane & 3));
+    const float f0 = __uint_as_float(w.x << 16), f1 = __uint_as_float(w.x & 0xffff0000u);
+    const float f2 = __uint_as_float(w.y << 16), f3 = __uint_as_float(w.y & 0xffff0000u);
+    qf[ks][0] = hv ? pack_f16x2(f0, f1) : 0u;
+    qf[ks][1] = hv ? pack_f16x2(f2, f3) : 0u;
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void load_q_frag(uint32_t (&qf)[D / 16][2], const __nv_bfloat16* q, int lane, int nh) {
   const int hn = lane >> 2;
@@ -346,8 +402,96 @@ __device__ __forceinline__ void warp_tile(WarpState<D>& st, const uint32_t (&qf)
   }
 }
 
-// Write one warp's state into the merge scratch (after a consumer barrier).
+// The 8-bit cache: one warp's 16 keys (kb .. kb+15) of the tile in `stage`
+// (codes), sk / sv the tile's K and V scales. Codes are exact in fp16: the
+// MMAs run fp16 x fp16 -> fp32, the K scale multiplies the score and the V
+// scale the probability (the softmax sums stay unscaled). A plain ldmatrix
+// gives a lane 4 consecutive codes of one key row: for Q K^T they are the
+// A operand with the head dims permuted as in load_q_frag_i8; for V^T P^T a
+// movmatrix transposes them into (dim, key pair) fragments, row m of a
+// 16-dim step d0 being dim d0 + i8_dim(m) (see stash_warp_state).
+__device__ __forceinline__ int i8_dim(int m) { return 4 * ((m & 7) >> 1) + (m & 1) + ((m >> 3) << 1); }
+
 template <int D>
+__device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&qf)[D / 16][2], uint32_t stage_addr,
+                                             const float* sk, const float* sv, int kb, int rows, int lane,
+                                             float scale_log2) {
+  using C = DecCfg<D, true>;
+  const uint32_t k_base = stage_addr;
+  const uint32_t v_base = stage_addr + C::kTileBytes;
+  // ldmatrix: matrices (rows 0-7, chunk c) (rows 8-15, chunk c) (rows 0-7, chunk c+1) (rows 8-15, chunk c+1)
+  const int row = kb + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int ch = lane >> 4;
+
+  // S^T = K * Q^T, two 16-dim steps per ldmatrix
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) {
+    uint32_t r0, r1, r2, r3;
+    ldmatrix_x4(k_base + sw128(row, 2 * j + ch), r0, r1, r2, r3);
+    uint32_t l0, h0, l1, h1, l2, h2, l3, h3;
+    int8x4_to_f16x2(r0, l0, h0);
+    int8x4_to_f16x2(r1, l1, h1);
+    int8x4_to_f16x2(r2, l2, h2);
+    int8x4_to_f16x2(r3, l3, h3);
+    mma_f16_16816(c, l0, l1, h0, h1, qf[2 * j][0], qf[2 * j][1]);
+    mma_f16_16816(c, l2, l3, h2, h3, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+  }
+
+  // online softmax (key kb + lane/4 in c0/c1, +8 in c2/c3), scores scaled by the key's K scale
+  const int key0 = kb + (lane >> 2);
+  const bool v0 = key0 < rows, v1 = key0 + 8 < rows;
+  const float s0 = v0 ? sk[key0] * scale_log2 : 0.f, s1 = v1 ? sk[key0 + 8] * scale_log2 : 0.f;
+  const float x0 = v0 ? c[0] * s0 : -INFINITY;
+  const float x1 = v0 ? c[1] * s0 : -INFINITY;
+  const float x2 = v1 ? c[2] * s1 : -INFINITY;
+  const float x3 = v1 ? c[3] * s1 : -INFINITY;
+  float mx_a = fmaxf(x0, x2), mx_b = fmaxf(x1, x3);
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+  }
+  const float mn_a = fmaxf(st.m_a, mx_a), mn_b = fmaxf(st.m_b, mx_b);
+  const float al_a = fast_exp2(st.m_a - mn_a), al_b = fast_exp2(st.m_b - mn_b);
+  st.m_a = mn_a;
+  st.m_b = mn_b;
+  const float p0 = fast_exp2(x0 - mn_a), p1 = fast_exp2(x1 - mn_b);
+  const float p2 = fast_exp2(x2 - mn_a), p3 = fast_exp2(x3 - mn_b);
+  st.l_a = st.l_a * al_a + p0 + p2;
+  st.l_b = st.l_b * al_b + p1 + p3;
+#pragma unroll
+  for (int md = 0; md < D / 16; ++md) {
+    st.o[md][0] *= al_a;
+    st.o[md][1] *= al_b;
+    st.o[md][2] *= al_a;
+    st.o[md][3] *= al_b;
+  }
+
+  // P^T times the V scales (keys past the valid rows: 0, their scales are never read)
+  const float w0 = v0 ? sv[key0] : 0.f, w1 = v1 ? sv[key0 + 8] : 0.f;
+  const uint32_t pb0 = movmatrix_trans(pack_f16x2(p0 * w0, p1 * w0));
+  const uint32_t pb1 = movmatrix_trans(pack_f16x2(p2 * w1, p3 * w1));
+
+  // O^T += V^T * P^T, two 16-dim steps per ldmatrix
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) {
+    uint32_t r0, r1, r2, r3;
+    ldmatrix_x4(v_base + sw128(row, 2 * j + ch), r0, r1, r2, r3);
+    uint32_t l0, h0, l1, h1, l2, h2, l3, h3;
+    int8x4_to_f16x2(r0, l0, h0);
+    int8x4_to_f16x2(r1, l1, h1);
+    int8x4_to_f16x2(r2, l2, h2);
+    int8x4_to_f16x2(r3, l3, h3);
+    mma_f16_16816(st.o[2 * j], movmatrix_trans(l0), movmatrix_trans(h0), movmatrix_trans(l1), movmatrix_trans(h1),
+                  pb0, pb1);
+    mma_f16_16816(st.o[2 * j + 1], movmatrix_trans(l2), movmatrix_trans(h2), movmatrix_trans(l3),
+                  movmatrix_trans(h3), pb0, pb1);
+  }
+}
+
+// Write one warp's state into the merge scratch (after a consumer barrier).
+template <int D, bool kInt8 = false>
 __device__ __forceinline__ void stash_warp_state(float* merge, const WarpState<D>& st, int warp, int lane) {
   float* red_m = merge;
   float* red_l = red_m + kDecConsumerWarps * kDecHeadsPerCta;
@@ -365,13 +509,16 @@ __device__ __forceinline__ void stash_warp_state(float* merge, const WarpState<D
     red_l[warp * 8 + ha] = l_a;
     red_l[warp * 8 + ha + 1] = l_b;
   }
+  // accumulator rows g and g + 8 of a 16-dim step: dims g and g + 8, or for
+  // the 8-bit path the dims its movmatrix fragments carry
   const int dr = lane >> 2;
+  const int da = kInt8 ? i8_dim(dr) : dr, db = kInt8 ? i8_dim(dr + 8) : dr + 8;
 #pragma unroll
   for (int md = 0; md < D / 16; ++md) {
-    ow[ha * D + md * 16 + dr] = st.o[md][0];
-    ow[(ha + 1) * D + md * 16 + dr] = st.o[md][1];
-    ow[ha * D + md * 16 + dr + 8] = st.o[md][2];
-    ow[(ha + 1) * D + md * 16 + dr + 8] = st.o[md][3];
+    ow[ha * D + md * 16 + da] = st.o[md][0];
+    ow[(ha + 1) * D + md * 16 + da] = st.o[md][1];
+    ow[ha * D + md * 16 + db] = st.o[md][2];
+    ow[(ha + 1) * D + md * 16 + db] = st.o[md][3];
   }
 }
 
@@ -476,12 +623,12 @@ __device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item)
 
 // End of a work item: merge the four warps, then write the output (a unit
 // with a single split) or the split's partial for decode_combine_kernel.
-template <int D>
+template <int D, bool kInt8 = false>
 __device__ __forceinline__ void item_epilogue(const DecodeParams& p, const ItemCoord& c, const WarpState<D>& st,
                                               float* merge, bool single, int tid, int warp, int lane) {
   __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(p.out) + ((size_t)c.b * p.H + c.h0) * D;
   consumer_bar();  // the previous epilogue has finished with the scratch
-  stash_warp_state<D>(merge, st, warp, lane);
+  stash_warp_state<D, kInt8>(merge, st, warp, lane);
   consumer_bar();
   const size_t part = ((size_t)c.unit * p.nsplit + c.split) * p.G + (size_t)c.hsl * kDecHeadsPerCta;
   for (int i = tid; i < c.nh * D; i += kDecConsumerWarps * 32) {
@@ -525,12 +672,17 @@ __device__ __forceinline__ void append_row(const DecodeParams& p, const ItemCoor
   __syncwarp();
 }
 
-template <int D, bool kPaged>
+// kPaged: the cache is a paged pool; kInt8: the cache holds 8-bit codes and
+// per-row scales (tm_k*/tm_v* then map codes, tm_ks/tm_vs the scales; the
+// bf16 kernels ignore tm_ks/tm_vs).
+template <int D, bool kPaged, bool kInt8>
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v64,
                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                        const DecodeParams p) {
-  using C = DecCfg<D>;
+  static_assert(!(kPaged && kInt8), "no paged 8-bit cache");
+  using C = DecCfg<D, kInt8>;
   extern __shared__ __align__(1024) uint8_t smem[];
   float* merge = reinterpret_cast<float*>(smem + C::kMergeOff);
   StageInfo* info = reinterpret_cast<StageInfo*>(smem + C::kInfoOff);
@@ -561,6 +713,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       prefetch_tensormap(&tm_v64);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
+      if constexpr (kInt8) {
+        prefetch_tensormap(&tm_ks);
+        prefetch_tensormap(&tm_vs);
+      }
       const uint64_t policy = l2_policy_evict_first();
       int it = 0;  // ring position
       bool ok = true;
@@ -609,6 +765,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           if constexpr (kPaged)
             issue_tile_paged<D>(smem + s * C::kStageBytes, &full[s], &tm_k64, &tm_v64, &tm_k, &tm_v, p, c.g, t0, blk,
                                 rows, policy);
+          else if constexpr (kInt8)
+            issue_tile_i8<D>(smem + s * C::kStageBytes, &full[s], &tm_k64, &tm_v64, &tm_k, &tm_v, &tm_ks, &tm_vs,
+                             c.unit * p.S_max + t0, c.unit, t0, rows, policy);
           else
             issue_tile<D>(smem + s * C::kStageBytes, &full[s], &tm_k64, &tm_v64, &tm_k, &tm_v, c.unit * p.S_max + t0,
                           rows, policy);
@@ -644,15 +803,30 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (si.item < 0) break;
     if (si.flags & kTileFirst) {
       cur = item_coord(p, si.item);
-      load_q_frag<D>(qf, static_cast<const __nv_bfloat16*>(p.q) + ((size_t)cur.b * p.H + cur.h0) * D, lane, cur.nh);
+      const __nv_bfloat16* qh = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)cur.b * p.H + cur.h0) * D;
+      if constexpr (kInt8)
+        load_q_frag_i8<D>(qf, qh, lane, cur.nh);
+      else
+        load_q_frag<D>(qf, qh, lane, cur.nh);
       st.reset();
     }
-    if (si.new_row >= 0 && (si.new_row >> 4) == warp)
-      append_row<D, kPaged>(p, cur, smem + s * C::kStageBytes, si.new_row, lane);
-    if (kb < si.rows) warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
+    if constexpr (!kInt8) {  // the fused append (bf16 caches only)
+      if (si.new_row >= 0 && (si.new_row >> 4) == warp)
+        append_row<D, kPaged>(p, cur, smem + s * C::kStageBytes, si.new_row, lane);
+    }
+    if (kb < si.rows) {
+      if constexpr (kInt8) {
+        const float* sk = reinterpret_cast<const float*>(smem + s * C::kStageBytes + C::kScaleOff);
+        warp_tile_i8<D>(st, qf, smem_u32(smem + s * C::kStageBytes), sk, sk + kDecTileKeys, kb, si.rows, lane,
+                        p.scale_log2);
+      } else {
+        warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
+      }
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-    if (si.flags & kTileLast) item_epilogue<D>(p, cur, st, merge, (si.flags & kUnitSingleSplit) != 0, tid, warp, lane);
+    if (si.flags & kTileLast)
+      item_epilogue<D, kInt8>(p, cur, st, merge, (si.flags & kUnitSingleSplit) != 0, tid, warp, lane);
   }
 }
 

@@ -81,6 +81,32 @@ bool encode_rows_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, 128] int8 codes, 128-byte rows (one swizzle span), box of box_rows rows.
+bool encode_rows_u8(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [units, S_max] float scales (row stride S_max * 4 bytes, a multiple of 16), box of 64 scales of one unit.
+bool encode_scales(CUtensorMap* map, const float* base, uint64_t units, uint64_t S_max) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {S_max, units};
+  cuuint64_t strides[1] = {S_max * 4};
+  cuuint32_t box[2] = {(cuuint32_t)gqa::kDecTileKeys, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int launch_status() { return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA; }
 
 // ----------------------------------------------------------------------------
@@ -144,14 +170,34 @@ int decode_ctas_per_sm(int dev) {
   if (cache[dev] == 0) {
     int n = 0;
     using C = gqa::DecCfg<D>;
-    if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<D, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(gqa::decode_bf16_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(gqa::decode_bf16_kernel<D, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_bf16_kernel<D, false>, gqa::kDecThreads,
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_bf16_kernel<D, false, false>, gqa::kDecThreads,
                                                       C::kSmemBytes) != cudaSuccess ||
         n <= 0) {
       cudaGetLastError();  // no GPU here: plan with the B200 figure
+      n = 2;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Resident 8-bit-cache decode CTAs per SM (2 on B200), cached per device.
+int decode_i8_ctas_per_sm(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return 2;
+  if (cache[dev] == 0) {
+    int n = 0;
+    using C = gqa::DecCfg<128, true>;
+    if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<128, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_bf16_kernel<128, false, true>,
+                                                      gqa::kDecThreads, C::kSmemBytes) != cudaSuccess ||
+        n <= 0) {
+      cudaGetLastError();
       n = 2;
     }
     cache[dev] = n;
@@ -180,10 +226,12 @@ int wide_ctas_per_sm(int dev) {
   return cache[dev];
 }
 
-DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gqa_dtype dt, int sms) {
+// int8: the 8-bit cache (narrow-group kernel only).
+DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gqa_dtype dt, int sms,
+                       bool int8 = false) {
   DecodePlan pl;
   const int G = H / K;
-  pl.wide = dt == GQA_BF16 && d == 128 && G % gqa::kWideHeads == 0;
+  pl.wide = !int8 && dt == GQA_BF16 && d == 128 && G % gqa::kWideHeads == 0;
   const int heads_per_cta =
       pl.wide ? gqa::kWideHeads : (dt == GQA_BF16 ? gqa::kDecHeadsPerCta : gqa::kDecF32HeadsPerCta);
   const int tile = pl.wide ? gqa::kWideKeys : 64;
@@ -212,8 +260,9 @@ DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gq
   if (dt == GQA_BF16) {
     // persistent CTAs that take work items from a counter in the workspace
     const int dev = current_device();
-    const int per_sm = pl.wide ? wide_ctas_per_sm(dev) : (d == 128 ? decode_ctas_per_sm<128>(dev)
-                                                                    : decode_ctas_per_sm<64>(dev));
+    const int per_sm = pl.wide ? wide_ctas_per_sm(dev)
+                               : int8 ? decode_i8_ctas_per_sm(dev)
+                                      : (d == 128 ? decode_ctas_per_sm<128>(dev) : decode_ctas_per_sm<64>(dev));
     const long long items = units * pl.nsplit;
     pl.grid = std::max<long long>(1, std::min<long long>(items, (long long)per_sm * sms));
     if (items + pl.grid >= (1ll << 24)) {  // beyond the work counter
@@ -240,12 +289,29 @@ int launch_decode_bf16(const DecodePlan& pl, const DecodeParams& p, const void* 
     return GQA_ERR_CUDA;
   using C = gqa::DecCfg<D>;
   decode_ctas_per_sm<D>(current_device());  // sets the shared-memory attribute once per device
+  // (the scale maps of the 8-bit kernel are unused here: the K maps stand in)
   if (p.block_table)
-    gqa::decode_bf16_kernel<D, true><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(tk64, tv64, tk, tv,
-                                                                                                p);
+    gqa::decode_bf16_kernel<D, true, false><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(
+        tk64, tv64, tk, tv, tk64, tv64, p);
   else
-    gqa::decode_bf16_kernel<D, false><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(tk64, tv64, tk, tv,
-                                                                                                 p);
+    gqa::decode_bf16_kernel<D, false, false><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(
+        tk64, tv64, tk, tv, tk64, tv64, p);
+  return launch_status();
+}
+
+// The 8-bit cache: codes [units * S_max, 128] int8, scales [units, S_max] float.
+int launch_decode_i8(const DecodePlan& pl, const DecodeParams& p, const void* kc, const void* vc, const float* ks,
+                     const float* vs, uint64_t units, uint64_t S_max, cudaStream_t st) {
+  CUtensorMap tk64, tv64, tk, tv, tks, tvs;
+  const uint64_t rows = units * S_max;
+  if (!encode_rows_u8(&tk64, kc, rows, gqa::kDecTileKeys) || !encode_rows_u8(&tv64, vc, rows, gqa::kDecTileKeys) ||
+      !encode_rows_u8(&tk, kc, rows, gqa::kDecBoxRows) || !encode_rows_u8(&tv, vc, rows, gqa::kDecBoxRows) ||
+      !encode_scales(&tks, ks, units, S_max) || !encode_scales(&tvs, vs, units, S_max))
+    return GQA_ERR_CUDA;
+  using C = gqa::DecCfg<128, true>;
+  decode_i8_ctas_per_sm(current_device());  // sets the shared-memory attribute once per device
+  gqa::decode_bf16_kernel<128, false, true><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(
+      tk64, tv64, tk, tv, tks, tvs, p);
   return launch_status();
 }
 
@@ -407,19 +473,24 @@ int kv_append_impl(void* k_cache, void* v_cache, const void* k_new, const void* 
 int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
                 int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
                 gqa_dtype dtype, gqa_stream_t stream, const void* k_new, const void* v_new, int append,
-                const PagedCache* pc = nullptr) {
+                const PagedCache* pc = nullptr, const float* k_scales = nullptr, const float* v_scales = nullptr) {
+  const bool int8 = k_scales != nullptr || v_scales != nullptr;  // caches of 8-bit codes with per-row scales
   if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
   if (num_splits < 0 || B < 0 || H <= 0 || K <= 0 || S_max <= 0) return GQA_ERR_INVALID_ARG;
   if (!valid_decode_shape(B, H, K, S_max, d, pc != nullptr)) return GQA_ERR_SHAPE;
   if (pc && !valid_paged(*pc, B, K)) return GQA_ERR_SHAPE;
   if (pc && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;  // the paged forms stream bf16 by TMA
+  if (int8 && (d != 128 || dtype != GQA_BF16 || pc || append)) return GQA_ERR_UNSUPPORTED;
+  if (int8 && S_max % 4 != 0) return GQA_ERR_SHAPE;  // a scale row must start on 16 bytes
   if (B == 0) return GQA_OK;
   if (!out || !q || !k_cache || !v_cache || !seqlens || (pc && !pc->table)) return GQA_ERR_INVALID_ARG;
+  if (int8 && (!k_scales || !v_scales)) return GQA_ERR_INVALID_ARG;
+  if (int8 && (!aligned16(k_scales) || !aligned16(v_scales))) return GQA_ERR_ALIGN;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return GQA_ERR_ALIGN;
   if (append && (!k_new || !v_new)) return GQA_ERR_INVALID_ARG;
   if (append && (!aligned16(k_new) || !aligned16(v_new))) return GQA_ERR_ALIGN;
   const int dev = current_device();
-  const DecodePlan pl = plan_decode(B, H, K, S_max, d, num_splits, dtype, sm_count(dev));
+  const DecodePlan pl = plan_decode(B, H, K, S_max, d, num_splits, dtype, sm_count(dev), int8);
   if (pl.ws_bytes == (size_t)-1) return GQA_ERR_SHAPE;  // more work items than the work counter holds
   if (pl.ws_bytes > 0) {
     if (!workspace || workspace_bytes < pl.ws_bytes) return GQA_ERR_INVALID_ARG;
@@ -464,7 +535,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.num_blocks = pc ? pc->num_blocks : 0;
   const uint64_t rows = pc ? (uint64_t)pc->num_blocks * K * pc->block_size : (uint64_t)B * K * S_max;
   int rc;
-  if (pl.wide)
+  if (int8)
+    rc = launch_decode_i8(pl, p, k_cache, v_cache, k_scales, v_scales, (uint64_t)B * K, (uint64_t)S_max, st);
+  else if (pl.wide)
     rc = launch_decode_wide(pl, p, q, k_cache, v_cache, B, H, rows, st);
   else if (dtype == GQA_BF16)
     rc = d == 128 ? launch_decode_bf16<128>(pl, p, k_cache, v_cache, rows, st)
@@ -549,6 +622,37 @@ int gqa_decode_append_paged(void* out, const void* q, void* k_pool, void* v_pool
   if (block_size <= 0 || max_blocks <= 0 || (long long)max_blocks * block_size >= (1ll << 31)) return GQA_ERR_SHAPE;
   return decode_impl(out, q, k_pool, v_pool, pos, B, H, K, max_blocks * block_size, d, scale, num_splits, workspace,
                      workspace_bytes, dtype, stream, k_new, v_new, 1, &pc);
+}
+
+int gqa_decode_int8(void* out, const void* q, const int8_t* k_codes, const float* k_scales, const int8_t* v_codes,
+                    const float* v_scales, const int32_t* seqlens, int B, int H, int K, int S_max, int d, float scale,
+                    int num_splits, void* workspace, size_t workspace_bytes, gqa_stream_t stream) {
+  if (!k_scales || !v_scales) return B == 0 ? GQA_OK : GQA_ERR_INVALID_ARG;
+  return decode_impl(out, q, k_codes, v_codes, seqlens, B, H, K, S_max, d, scale, num_splits, workspace,
+                     workspace_bytes, GQA_BF16, stream, nullptr, nullptr, 0, nullptr, k_scales, v_scales);
+}
+
+size_t gqa_decode_int8_workspace_bytes(int B, int H, int K, int S_max, int d, int num_splits) {
+  if (!valid_decode_shape(B, H, K, S_max, d) || d != 128 || S_max % 4 != 0 || num_splits < 0) return 0;
+  const DecodePlan a = plan_decode(B, H, K, S_max, d, num_splits, GQA_BF16, sm_count(current_device()), true);
+  if (a.ws_bytes == (size_t)-1) return 0;
+  return a.ws_bytes;
+}
+
+int gqa_kv_append_int8(int8_t* k_codes, float* k_scales, int8_t* v_codes, float* v_scales, const void* k_new,
+                       const void* v_new, const int32_t* pos, int B, int K, int S_max, int d, gqa_stream_t stream) {
+  if (B < 0 || K <= 0 || S_max <= 0) return GQA_ERR_INVALID_ARG;
+  if (d != 128) return GQA_ERR_UNSUPPORTED;
+  if (B == 0) return GQA_OK;
+  if (!k_codes || !k_scales || !v_codes || !v_scales || !k_new || !v_new || !pos) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_new) || !aligned16(v_new)) return GQA_ERR_ALIGN;
+  const long long warps = 2ll * B * K;
+  const int dev = current_device();
+  const int grid = grid_for(warps * 32, 256, sm_count(dev));
+  gqa::kv_append_int8_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
+      k_codes, k_scales, v_codes, v_scales, static_cast<const __nv_bfloat16*>(k_new),
+      static_cast<const __nv_bfloat16*>(v_new), pos, B, K, S_max);
+  return launch_status();
 }
 
 size_t gqa_decode_paged_workspace_bytes(int B, int H, int K, int d, int block_size, int max_blocks, int num_splits) {

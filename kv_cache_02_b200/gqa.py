@@ -29,6 +29,7 @@ GQA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode", "gqa_decode_append", "gqa_decode_noalloc",
             "gqa_decode_paged_workspace_bytes", "gqa_decode_paged", "gqa_decode_append_paged", "gqa_kv_append_paged",
+            "gqa_decode_int8_workspace_bytes", "gqa_decode_int8", "gqa_kv_append_int8",
             "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string")
 
 
@@ -62,6 +63,12 @@ def _load():
     lib.gqa_decode_append_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P, SZ, I, P]
     lib.gqa_kv_append_paged.restype = I
     lib.gqa_kv_append_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P]
+    lib.gqa_decode_int8_workspace_bytes.restype = SZ
+    lib.gqa_decode_int8_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.gqa_decode_int8.restype = I
+    lib.gqa_decode_int8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, P]
+    lib.gqa_kv_append_int8.restype = I
+    lib.gqa_kv_append_int8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P]
     lib.gqa_prefill_causal.restype = I
     lib.gqa_prefill_causal.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gqa_meanpool_kv.restype = I
@@ -217,6 +224,35 @@ def gqa_kv_append_paged(k_pool, v_pool, k_new, v_new, block_table, pos, stream=N
            _lib.gqa_kv_append_paged(_ptr(k_pool), _ptr(v_pool), _ptr(k_new), _ptr(v_new), _ptr(block_table),
                                     _ptr(pos), B, K, d, num_blocks, block_size, block_table.shape[1],
                                     _dtype(k_pool), _stream(stream)))
+
+
+def gqa_decode_int8_workspace_bytes(B: int, H: int, K: int, S_max: int, d: int, num_splits: int = 0) -> int:
+    return int(_lib.gqa_decode_int8_workspace_bytes(B, H, K, S_max, d, num_splits))
+
+
+def gqa_decode_int8(out, q, k_codes, k_scales, v_codes, v_scales, seqlens, scale: float, num_splits: int = 0,
+                    workspace=None, stream=None) -> None:
+    """out/q [B,H,d] bf16; codes [B,K,S_max,d] int8; scales [B,K,S_max] float32; seqlens [B] int32."""
+    B, H, d = q.shape
+    _, K, S_max, _ = k_codes.shape
+    assert out.shape == q.shape and q.dtype == torch.bfloat16 and k_codes.dtype == torch.int8
+    assert v_codes.shape == k_codes.shape and v_codes.dtype == torch.int8
+    assert k_scales.shape == (B, K, S_max) and v_scales.shape == k_scales.shape and k_scales.dtype == torch.float32
+    assert seqlens.dtype == torch.int32 and seqlens.shape == (B,)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("gqa_decode_int8", _lib.gqa_decode_int8(_ptr(out), _ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                                                   _ptr(v_scales), _ptr(seqlens), B, H, K, S_max, d, float(scale),
+                                                   int(num_splits), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def gqa_kv_append_int8(k_codes, k_scales, v_codes, v_scales, k_new, v_new, pos, stream=None) -> None:
+    """Quantize k_new/v_new [B,K,d] bf16 into the 8-bit caches at key pos[b] (codes and scales in place)."""
+    B, K, S_max, d = k_codes.shape
+    assert k_new.shape == (B, K, d) and v_new.shape == (B, K, d) and k_new.dtype == torch.bfloat16
+    assert pos.dtype == torch.int32 and pos.shape == (B,)
+    _check("gqa_kv_append_int8", _lib.gqa_kv_append_int8(_ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                                                         _ptr(v_scales), _ptr(k_new), _ptr(v_new), _ptr(pos), B, K,
+                                                         S_max, d, _stream(stream)))
 
 
 def gqa_prefill_causal(out, q, k, v, scale: float, k_cache=None, v_cache=None, stream=None) -> None:

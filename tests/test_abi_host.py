@@ -30,7 +30,9 @@ def test_header_declares_the_boundary():
     assert declared_symbols() == sorted(["gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode",
                                          "gqa_decode_append", "gqa_decode_noalloc",
                                          "gqa_decode_paged_workspace_bytes", "gqa_decode_paged",
-                                         "gqa_decode_append_paged", "gqa_kv_append_paged", "gqa_prefill_causal",
+                                         "gqa_decode_append_paged", "gqa_kv_append_paged",
+                                         "gqa_decode_int8_workspace_bytes", "gqa_decode_int8", "gqa_kv_append_int8",
+                                         "gqa_prefill_causal",
                                          "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string"])
 
 
@@ -115,6 +117,25 @@ def test_paged_calls_reject_bad_arguments(lib):
     ws = lib.gqa_decode_paged_workspace_bytes
     assert ws(1, 8, 2, 64, 24, 8, 0) == 0 and ws(1, 6, 4, 64, 16, 8, 0) == 0
     assert ws(1, 64, 8, 128, 16, 8192, 0) > 0  # a long sequence is split
+
+
+def test_int8_calls_reject_bad_arguments(lib):
+    f = lib.gqa_decode_int8
+    # out, q, k_codes, k_scales, v_codes, v_scales, seqlens, B, H, K, S_max, d, scale, splits, ws, ws_bytes, stream
+    assert f(P, P, P, P, P, P, P, 2, 8, 2, 64, 64, 1.0, 0, None, 0, None) == -6     # head dim 64
+    assert f(P, P, P, P, P, P, P, 2, 8, 2, 66, 128, 1.0, 0, None, 0, None) == -2    # S_max not a multiple of 4
+    assert f(P, P, P, P, P, P, P, 2, 6, 4, 64, 128, 1.0, 0, None, 0, None) == -2    # H % K != 0
+    assert f(P, P, P, None, P, P, P, 2, 8, 2, 64, 128, 1.0, 0, None, 0, None) == -1  # no scales
+    assert f(P, P, P, P + 4, P, P, P, 2, 8, 2, 64, 128, 1.0, 0, None, 0, None) == -3  # misaligned scales
+    assert f(P, P, P, P, P, P, P, 1, 8, 2, 1 << 14, 128, 1.0, 0, None, 0, None) == -1  # split plan, no workspace
+    assert f(None, None, None, P, None, P, None, 0, 8, 2, 64, 128, 1.0, 0, None, 0, None) == 0
+    a = lib.gqa_kv_append_int8
+    assert a(P, P, P, P, P, P, P, 2, 2, 64, 64, None) == -6
+    assert a(P, None, P, P, P, P, P, 2, 2, 64, 128, None) == -1
+    assert a(None, None, None, None, None, None, None, 0, 2, 64, 128, None) == 0
+    ws = lib.gqa_decode_int8_workspace_bytes
+    assert ws(1, 8, 2, 64, 64, 0) == 0 and ws(1, 8, 2, 66, 128, 0) == 0
+    assert ws(1, 64, 8, 131072, 128, 0) > 0
 
 
 def test_prefill_rejects_bad_arguments(lib):
