@@ -27,6 +27,10 @@ Page citations (title, section):
     head), value = code * scale; quantization in float32: scale = amax / 127,
     code = round-half-even(x / scale). Decoding an 8-bit cache is the decode
     of the values it holds.
+  * Varlen prefill: "GQA 完全拆解", section 主流模型里的 GQA：KV 缓存账本
+    (continuous batching with the KV cache: requests of different lengths
+    batched together); each sequence of a packed batch is prefilled causally
+    on its own.
   * Paged KV cache: "分組查詢注意力", section 下游 / 推論引擎與架構 (the
     paged cache manages blocks of the K KV heads, not of the H query heads,
     and each block is broadcast to the group's H/K query heads when it is
@@ -373,3 +377,34 @@ def kv_append_int8(k_codes, k_scales, v_codes, v_scales, k_new, v_new, pos, lib=
             kc[b, :, p], ks[b, :, p] = kq[b], kqs[b]
             vc[b, :, p], vs[b, :, p] = vq[b], vqs[b]
     return kc, ks, vc, vs
+
+
+# ---------------------------------------------------------------------------
+# varlen (packed) causal prefill: the sequences of a continuous batch back to back
+
+def prefill_causal_varlen(q, k, v, cu_seqlens, scale: float, nthreads=None, lib=None) -> np.ndarray:
+    """q [T,H,d], k/v [T,K,d] holding B sequences back to back, sequence b being tokens
+    cu_seqlens[b] .. cu_seqlens[b+1]-1 -> float64 [T,H,d]: the causal prefill of every sequence on
+    its own (a token sees the keys of its own sequence up to itself)."""
+    q, k, v = _c(q), _c(k), _c(v)
+    T, H, d = q.shape
+    out = np.zeros((T, H, d), dtype=np.float64)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    for b in range(len(cu) - 1):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        if s1 > s0:
+            out[s0:s1] = prefill_causal(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], scale, nthreads=nthreads,
+                                        lib=lib)[0]
+    return out
+
+
+def prefill_cache_write_varlen(k, v, cu_seqlens, S_max: int, k_cache, v_cache):
+    """k/v [T,K,d] packed -> copies of the caches [B,K,S_max,d] with rows 0..len_b-1 of sequence b set."""
+    kc, vc = np.array(k_cache, copy=True), np.array(v_cache, copy=True)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    for b in range(len(cu) - 1):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        n = min(s1 - s0, S_max)
+        kc[b, :, :n, :] = np.transpose(k[s0:s0 + n], (1, 0, 2))
+        vc[b, :, :n, :] = np.transpose(v[s0:s0 + n], (1, 0, 2))
+    return kc, vc

@@ -314,3 +314,35 @@ def int8_inputs(name: str) -> dict:
     return {"q": normal((w.B, w.H, w.d), BF16, w.seed, STREAM_Q), "k_codes": kc.reshape(*shp, w.d),
             "k_scale": ks.reshape(shp), "v_codes": vc.reshape(*shp, w.d), "v_scale": vs.reshape(shp),
             "seqlens": lens}
+
+
+# --------------------------------------------------------------------------
+# varlen prefill: a continuous batch of prompts of different lengths, packed
+
+
+@dataclasses.dataclass(frozen=True)
+class VarlenShape:
+    name: str
+    B: int
+    H: int
+    K: int
+    d: int
+    len_range: tuple  # prompt lengths uniform in [lo, hi]
+    S_max: int        # cache capacity per sequence
+    seed: int
+
+
+VARLEN_WORKLOADS = {
+    "varlen_prefill_b8_h32_k8_d128_s256_4k": VarlenShape(
+        "varlen_prefill_b8_h32_k8_d128_s256_4k", 8, 32, 8, 128, (256, 4096), 4096, SEED_BASE + 5),
+}
+
+
+def varlen_inputs(w: VarlenShape) -> dict:
+    """lens [B], cu_seqlens [B+1], q [T,H,d], k/v [T,K,d] (bf16, T = sum of lens)."""
+    lens = uniform_int(w.B, w.len_range[0], w.len_range[1], w.seed, STREAM_LENS)
+    cu = np.zeros(w.B + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lens)
+    T = int(cu[-1])
+    return {"lens": lens, "cu_seqlens": cu, "q": normal((T, w.H, w.d), BF16, w.seed, STREAM_Q),
+            "k": normal((T, w.K, w.d), BF16, w.seed, STREAM_K), "v": normal((T, w.K, w.d), BF16, w.seed, STREAM_V)}
