@@ -292,6 +292,7 @@ DECODE_EXTRA = ["ragged_70b_decode_b32_h64_k8_d128_s1k_16k", "long_ctx_gqa_b1_h6
 PREFILL = "causal_prefill_b4_s4096_h32_k8_d128"
 PAGED_EXTRA = list(synth.PAGED_WORKLOADS)
 INT8_EXTRA = list(synth.INT8_WORKLOADS)
+VARLEN_EXTRA = list(synth.VARLEN_WORKLOADS)
 
 
 class L2Flush:
@@ -359,6 +360,10 @@ def extra_measurements(args, only=None):
         if only is not None and name != only:
             continue
         res[name] = int8_measurement(args, name, peaks, 20 if only is None else args.steps)
+    for name in VARLEN_EXTRA:
+        if only is not None and name != only:
+            continue
+        res[name] = varlen_measurement(args, name, peaks, 20 if only is None else args.steps)
     if only is not None and only != PREFILL:
         return res
     # causal prefill with the KV-cache write: FLOPs over the causal pairs (j <= i) only
@@ -492,6 +497,46 @@ def int8_measurement(args, name, peaks, steps):
     return r
 
 
+def varlen_measurement(args, name, peaks, steps):
+    """gqa_prefill_causal_varlen (with the cache write): FLOPs over every sequence's causal pairs."""
+    import torch
+
+    from kv_cache_02_b200 import gqa
+
+    w = synth.VARLEN_WORKLOADS[name]
+    inp = synth.varlen_inputs(w)
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).cuda()
+
+    q, k, v, cu = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), to_dev(inp["cu_seqlens"])
+    out = torch.empty_like(q)
+    kc = torch.empty((w.B, w.K, w.S_max, w.d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    lens = inp["lens"].astype(np.float64)
+    flops = float(np.sum(4.0 * w.H * w.d * lens * (lens + 1) / 2))
+    times = []
+    for it in range(args.warmup + steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        gqa.gqa_prefill_causal_varlen(out, q, k, v, cu, 1.0 / np.sqrt(w.d), kc, vc)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            times.append(a.elapsed_time(b))
+    if gqa.gqa_get_last_error() != (0, 0):
+        raise RuntimeError(f"device error in {name}")
+    ms = statistics.median(times)
+    tf = flops / (ms * 1e-3) / 1e12
+    r = {"ms": round(ms, 4), "flops": flops, "TFLOP/s": round(tf, 1), "tokens": int(lens.sum()),
+         "frac_of_measured_bf16_burst": round(tf / peaks["bf16_tflops"], 4),
+         "includes": "attention + KV-cache write"}
+    del q, k, v, cu, out, kc, vc
+    torch.cuda.empty_cache()
+    return r
+
+
 def cpu_baseline(inp, scale, kv_bytes_layer):
     """The oracle as it stands, on all host cores, over one full layer of the workload."""
     import oracle
@@ -546,7 +591,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads and the CPU baseline")
-    ap.add_argument("--only", choices=DECODE_EXTRA + PAGED_EXTRA + INT8_EXTRA + [PREFILL], default=None,
+    ap.add_argument("--only", choices=DECODE_EXTRA + PAGED_EXTRA + INT8_EXTRA + VARLEN_EXTRA + [PREFILL],
+                    default=None,
                     help="time one other workload alone (for profiling); prints its own JSON, not the contract line")
     ap.add_argument("--layers", type=int, default=32,
                     help="layers per step (32 for the model; fewer only for small profiling captures)")

@@ -288,6 +288,26 @@ GQA_API int gqa_prefill_causal(void* out, const void* q, const void* k, const vo
                        int S, int H, int K, int S_max, int d, float scale, gqa_dtype dtype, gqa_stream_t stream);
 
 /*
+ * gqa_prefill_causal_varlen - gqa_prefill_causal over a packed batch of
+ * prompts of different lengths (continuous batching, "GQA 完全拆解", section
+ * 主流模型里的 GQA：KV 缓存账本): every sequence is prefilled causally on its own.
+ *
+ * q, out     : [T, H, d]; k, v : [T, K, d]: the B sequences back to back.
+ * cu_seqlens : [B + 1] int32, device: sequence b is rows cu_seqlens[b] ..
+ *              cu_seqlens[b+1] - 1 (cu_seqlens[0] = 0, nondecreasing,
+ *              cu_seqlens[B] = T). Entries outside [0, T] or decreasing set
+ *              GQA_DEVERR_SEQLEN and are clamped into [0, T].
+ * k_cache,
+ * v_cache    : [B, K, S_max, d] or both NULL. When given, row t of sequence b
+ *              is written at key t; rows at or past S_max are not written
+ *              and set GQA_DEVERR_SEQLEN.
+ * dtype      : GQA_BF16 only (GQA_F32 returns GQA_ERR_UNSUPPORTED).
+ */
+GQA_API int gqa_prefill_causal_varlen(void* out, const void* q, const void* k, const void* v, void* k_cache,
+                                      void* v_cache, const int32_t* cu_seqlens, int B, int T, int H, int K,
+                                      int S_max, int d, float scale, gqa_dtype dtype, gqa_stream_t stream);
+
+/*
  * gqa_meanpool_kv - MHA -> GQA conversion by mean pooling of heads.
  *
  * "分組查詢注意力", section 模型轉換與 Uptraining, and "GQA 完全拆解", section

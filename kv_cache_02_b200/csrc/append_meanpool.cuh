@@ -115,6 +115,43 @@ __global__ void kv_write_prompt_kernel(uint4* __restrict__ k_cache, uint4* __res
   }
 }
 
+// Varlen prompt write: packed k [T, K, d] of B sequences (cu_seqlens) ->
+// k_cache [B, K, S_max, d], row t of sequence b at key t (and V). A token's
+// sequence is found by binary search in cu_seqlens; rows at or past S_max
+// are not written and set GQA_DEVERR_SEQLEN.
+__global__ void kv_write_prompt_varlen_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                                              const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                              const int32_t* __restrict__ cu_seqlens, int B, int T, int K, int S_max,
+                                              int chunks_per_row) {
+  const long long per_tensor = (long long)T * K * chunks_per_row;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < 2 * per_tensor;
+       i += (long long)gridDim.x * blockDim.x) {
+    const bool is_v = i >= per_tensor;
+    const long long j = is_v ? i - per_tensor : i;  // index in [T, K, chunks]
+    const int c = (int)(j % chunks_per_row);
+    const long long r = j / chunks_per_row;
+    const int g = (int)(r % K);
+    const int t = (int)(r / K);
+    int lo = 0, hi = B;  // the sequence b with cu[b] <= t < cu[b+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(cu_seqlens + mid) <= t) lo = mid;
+      else hi = mid;
+    }
+    const int pos = t - __ldg(cu_seqlens + lo);
+    if (pos < 0 || t >= __ldg(cu_seqlens + lo + 1)) continue;  // a token outside every sequence
+    if (pos >= S_max) {
+      if (c == 0 && g == 0 && !is_v) raise_error(GQA_DEVERR_SEQLEN);
+      continue;
+    }
+    const long long dst = (((long long)lo * K + g) * S_max + pos) * chunks_per_row + c;
+    if (is_v)
+      v_cache[dst] = __ldg(v + j);
+    else
+      k_cache[dst] = __ldg(k + j);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // gqa_meanpool_kv: dst[o, g, i] = sum_{r<G} src[o, g*G + r, i] / G.
 // The sum runs in double in ascending r and is rounded once to the output

@@ -368,6 +368,23 @@ int launch_prefill(void* out, const void* q, const void* k, const void* v, void*
   return launch_status();
 }
 
+// Varlen: packed [T, heads, d] tokens of B sequences given by cu_seqlens.
+int launch_prefill_varlen(void* out, const void* q, const void* k, const void* v, void* k_cache, void* v_cache,
+                          const int32_t* cu_seqlens, int B, int T, int H, int K, int S_max, int d, float scale,
+                          cudaStream_t st, int sms) {
+  auto fn = reinterpret_cast<gqa::PfEncodeFn>(encode_fn());
+  if (!fn) return GQA_ERR_CUDA;
+  int rc = d == 128 ? gqa::launch_prefill_d<128>(fn, out, q, k, v, B, 0, H, K, scale, st, cu_seqlens, T)
+                    : gqa::launch_prefill_d<64>(fn, out, q, k, v, B, 0, H, K, scale, st, cu_seqlens, T);
+  if (rc != GQA_OK || !k_cache) return rc;
+  const int cpr = d * 2 / 16;
+  const long long work = 2ll * T * K * cpr;
+  gqa::kv_write_prompt_varlen_kernel<<<grid_for(work, 256, sms), 256, 0, st>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
+      static_cast<const uint4*>(v), cu_seqlens, B, T, K, S_max, cpr);
+  return launch_status();
+}
+
 }  // namespace
 
 // ============================================================================
@@ -680,6 +697,25 @@ int gqa_prefill_causal(void* out, const void* q, const void* k, const void* v, v
   if (dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
   return launch_prefill(out, q, k, v, k_cache, v_cache, B, S, H, K, S_max, d, scale, (cudaStream_t)stream,
                         sm_count(current_device()));
+}
+
+int gqa_prefill_causal_varlen(void* out, const void* q, const void* k, const void* v, void* k_cache, void* v_cache,
+                              const int32_t* cu_seqlens, int B, int T, int H, int K, int S_max, int d, float scale,
+                              gqa_dtype dtype, gqa_stream_t stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (B < 0 || T < 0 || H <= 0 || K <= 0) return GQA_ERR_INVALID_ARG;
+  if (H % K != 0 || (d != 64 && d != 128)) return GQA_ERR_SHAPE;
+  if (dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
+  if ((k_cache == nullptr) != (v_cache == nullptr)) return GQA_ERR_INVALID_ARG;
+  if (k_cache && S_max <= 0) return GQA_ERR_INVALID_ARG;
+  if ((long long)T + 128ll * (B + 1) >= (1ll << 31)) return GQA_ERR_SHAPE;  // TMA row coordinates are int32
+  if (((long long)T / 128 + B + 1) * H >= (1ll << 31)) return GQA_ERR_SHAPE;
+  if (B == 0 || T == 0) return GQA_OK;
+  if (!out || !q || !k || !v || !cu_seqlens) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return GQA_ERR_ALIGN;
+  if (k_cache && (!aligned16(k_cache) || !aligned16(v_cache))) return GQA_ERR_ALIGN;
+  return launch_prefill_varlen(out, q, k, v, k_cache, v_cache, cu_seqlens, B, T, H, K, S_max, d, scale,
+                               (cudaStream_t)stream, sm_count(current_device()));
 }
 
 int gqa_meanpool_kv(void* dst, const void* src, int64_t outer, int H, int K, int64_t inner, gqa_dtype dtype,

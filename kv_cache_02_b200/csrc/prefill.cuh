@@ -48,16 +48,20 @@ struct PfCfg {
   static constexpr int kBarOff = kPOff + kPBytes;
   static constexpr int kNumBars = 1 + 4 * kPfStages + 2 + 2 + 1 + 1 + 1;
   // at most two CTAs per SM (their 2 x 256 TMEM columns fill the SM's 512)
-  static constexpr int kSmemBytes = (kBarOff + kNumBars * 8 + 16) > 80 * 1024 ? (kBarOff + kNumBars * 8 + 16)
+  static constexpr int kSmemBytes = (kBarOff + kNumBars * 8 + 32) > 80 * 1024 ? (kBarOff + kNumBars * 8 + 32)
                                                                                : 80 * 1024;
   static constexpr int kOCol = 2 * kPfBN;  // TMEM column of O (after the two S buffers)
   static_assert(kOCol + D <= kPfTmemCols, "TMEM budget");
 };
 
 struct PrefillParams {
-  void* out;  // [B, S, H, D] bf16
+  void* out;  // [B, S, H, D] bf16, or packed [T, H, D] with cu_seqlens
   int B, S, H, K, G, n_qt;
   float scale_log2;
+  // varlen (a packed continuous batch): sequence b is tokens cu_seqlens[b] ..
+  // cu_seqlens[b+1]-1 of the T rows; null for the fixed-length [B, S] layout
+  const int32_t* cu_seqlens;
+  int T;
 };
 
 template <int D>
@@ -87,14 +91,60 @@ __global__ void __launch_bounds__(kPfThreads, 2)
     return;
   }
 
-  // work item: heavy query tiles first; the G heads of a group are adjacent
-  const int per_qt = p.B * p.H;
-  const int qt = p.n_qt - 1 - (int)(blockIdx.x / per_qt);
-  const int rem = (int)(blockIdx.x % per_qt);
-  const int b = rem / p.H, h = rem % p.H;
+  // work item (query tile qt of sequence b, head h): rows seq0 .. seq0+len-1.
+  // Fixed length: heavy query tiles first, the G heads of a group adjacent.
+  // Varlen: tiles sequence by sequence, each sequence's heaviest first, the
+  // heads of a tile adjacent; thread 0 finds the tile's sequence (the grid is
+  // sized for the worst case, and CTAs past the last tile end here).
+  int qt, b, h, seq0, len;
+  if (p.cu_seqlens == nullptr) {
+    const int per_qt = p.B * p.H;
+    qt = p.n_qt - 1 - (int)(blockIdx.x / per_qt);
+    const int rem = (int)(blockIdx.x % per_qt);
+    b = rem / p.H;
+    h = rem % p.H;
+    seq0 = b * p.S;
+    len = p.S;
+  } else {
+    int* s_item = reinterpret_cast<int*>(smem + C::kBarOff + C::kNumBars * 8 + 8);
+    h = (int)(blockIdx.x % p.H);
+    const int t_idx = (int)(blockIdx.x / p.H);
+    if (threadIdx.x == 0) {
+      // sequence by sequence, each sequence's heaviest tile first (measured
+      // faster than ordering all sequences' tiles by weight: a sequence's K/V
+      // tiles stay hot in L2 while its query tiles run)
+      int acc = 0, fb = -1, fs0 = 0, flen = 0, fqt = 0;
+      bool bad = false;
+      for (int bb = 0; bb < p.B; ++bb) {
+        int s0 = __ldg(p.cu_seqlens + bb), s1 = __ldg(p.cu_seqlens + bb + 1);
+        if (s0 < 0 || s1 > p.T || s1 < s0) bad = true;  // clamped to the packed rows
+        s0 = min(max(s0, 0), p.T);
+        s1 = min(max(s1, s0), p.T);
+        const int n = (s1 - s0 + kPfBM - 1) / kPfBM;
+        if (fb < 0 && t_idx < acc + n) {
+          fb = bb;
+          fs0 = s0;
+          flen = s1 - s0;
+          fqt = n - 1 - (t_idx - acc);
+        }
+        acc += n;
+      }
+      if (bad && blockIdx.x == 0) raise_error(GQA_DEVERR_SEQLEN);
+      s_item[0] = fb;
+      s_item[1] = fs0;
+      s_item[2] = flen;
+      s_item[3] = fqt;
+    }
+    __syncthreads();
+    b = s_item[0];
+    seq0 = s_item[1];
+    len = s_item[2];
+    qt = s_item[3];
+    if (b < 0) return;
+  }
   const int g = h / p.G;
   const int q0 = qt * kPfBM;
-  const int n_tiles = min((p.S + kPfBN - 1) / kPfBN, (q0 + kPfBM + kPfBN - 1) / kPfBN);
+  const int n_tiles = min((len + kPfBN - 1) / kPfBN, (q0 + kPfBM + kPfBN - 1) / kPfBN);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -140,7 +190,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
         mbar_arrive_expect_tx(q_full, C::kQBytes);
 #pragma unroll
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_3d(smem + C::kQOff + hf * C::kQHalf, &tm_q, hf * 64, h, b * p.S + q0, q_full, pol_q);
+          tma_load_3d(smem + C::kQOff + hf * C::kQHalf, &tm_q, hf * 64, h, seq0 + q0, q_full, pol_q);
       }
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
@@ -150,7 +200,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
         mbar_arrive_expect_tx(&full[s], C::kTileBytes);
 #pragma unroll
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_3d(dst + hf * C::kKVHalf, tm, hf * 64, g, b * p.S + j * kPfBN, &full[s], pol_kv);
+          tma_load_3d(dst + hf * C::kKVHalf, tm, hf * 64, g, seq0 + j * kPfBN, &full[s], pol_kv);
         ++issued;
       }
       for (int j = max(0, issued - kPfStages); j < issued; ++j)
@@ -236,7 +286,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
       mbar_arrive(&s_free[j & 1]);
 
       const int k0 = j * kPfBN;
-      const int kmax = min(qpos, p.S - 1) - k0;  // keys k0 + c with c <= kmax are visible
+      const int kmax = min(qpos, len - 1) - k0;  // keys k0 + c with c <= kmax are visible
       // With a positive scale the maximum is taken on the raw scores and the
       // scale folds into the exponent (one FFMA per score); off-diagonal
       // tiles need no mask.
@@ -307,13 +357,13 @@ __global__ void __launch_bounds__(kPfThreads, 2)
       tc_fence_after();
       const float inv_l = 1.f / l;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-      uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)b * p.S + qpos) * p.H + h) * D);
+      uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)seq0 + qpos) * p.H + h) * D);
 #pragma unroll 1
       for (int cb = 0; cb < D; cb += 32) {
         float o[32];
         tmem_ld32(lane_addr + C::kOCol + cb, o);
         tc_wait_ld();
-        if (qpos < p.S) {
+        if (qpos < len) {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             dst[cb / 8 + i] = make_uint4(pack_bf16x2(o[8 * i] * inv_l, o[8 * i + 1] * inv_l),
@@ -351,13 +401,18 @@ inline bool encode_bsh(PfEncodeFn fn, CUtensorMap* map, const void* base, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Fixed length: q/out [B, S, H, D], k/v [B, S, K, D] (cu_seqlens null).
+// Varlen: packed q/out [T, H, D], k/v [T, K, D], B sequences given by
+// cu_seqlens (device); S is unused and the grid covers the worst case of
+// ceil(T / 128) + B query tiles per head.
 template <int D>
 int launch_prefill_d(PfEncodeFn fn, void* out, const void* q, const void* k, const void* v, int B, int S, int H,
-                     int K, float scale, cudaStream_t st) {
+                     int K, float scale, cudaStream_t st, const int32_t* cu_seqlens = nullptr, int T = 0) {
   using C = PfCfg<D>;
   CUtensorMap tq, tk, tv;
-  if (!encode_bsh(fn, &tq, q, (uint64_t)B * S, H, D, kPfBM) || !encode_bsh(fn, &tk, k, (uint64_t)B * S, K, D, kPfBN) ||
-      !encode_bsh(fn, &tv, v, (uint64_t)B * S, K, D, kPfBN))
+  const uint64_t rows = cu_seqlens ? (uint64_t)T : (uint64_t)B * S;
+  if (!encode_bsh(fn, &tq, q, rows, H, D, kPfBM) || !encode_bsh(fn, &tk, k, rows, K, D, kPfBN) ||
+      !encode_bsh(fn, &tv, v, rows, K, D, kPfBN))
     return GQA_ERR_CUDA;
   static bool configured[64] = {false};
   int dev = 0;
@@ -377,7 +432,9 @@ int launch_prefill_d(PfEncodeFn fn, void* out, const void* q, const void* k, con
   p.G = H / K;
   p.n_qt = (S + kPfBM - 1) / kPfBM;
   p.scale_log2 = scale * 1.4426950408889634f;
-  const long long grid = (long long)p.n_qt * B * H;
+  p.cu_seqlens = cu_seqlens;
+  p.T = T;
+  const long long grid = cu_seqlens ? ((long long)(T + kPfBM - 1) / kPfBM + B) * H : (long long)p.n_qt * B * H;
   prefill_causal_kernel<D><<<(unsigned)grid, kPfThreads, C::kSmemBytes, st>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }

@@ -29,7 +29,7 @@ GQA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode", "gqa_decode_append", "gqa_decode_noalloc",
             "gqa_decode_paged_workspace_bytes", "gqa_decode_paged", "gqa_decode_append_paged", "gqa_kv_append_paged",
-            "gqa_decode_int8_workspace_bytes", "gqa_decode_int8", "gqa_kv_append_int8",
+            "gqa_decode_int8_workspace_bytes", "gqa_decode_int8", "gqa_kv_append_int8", "gqa_prefill_causal_varlen",
             "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string")
 
 
@@ -71,6 +71,8 @@ def _load():
     lib.gqa_kv_append_int8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P]
     lib.gqa_prefill_causal.restype = I
     lib.gqa_prefill_causal.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.gqa_prefill_causal_varlen.restype = I
+    lib.gqa_prefill_causal_varlen.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gqa_meanpool_kv.restype = I
     lib.gqa_meanpool_kv.argtypes = [P, P, I64, I, I, I64, I, P]
     lib.gqa_get_last_error.restype = I
@@ -266,6 +268,22 @@ def gqa_prefill_causal(out, q, k, v, scale: float, k_cache=None, v_cache=None, s
     _check("gqa_prefill_causal", _lib.gqa_prefill_causal(_ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache),
                                                          _ptr(v_cache), B, S, H, K, S_max, d, float(scale),
                                                          _dtype(q), _stream(stream)))
+
+
+def gqa_prefill_causal_varlen(out, q, k, v, cu_seqlens, scale: float, k_cache=None, v_cache=None,
+                              stream=None) -> None:
+    """Packed out/q [T,H,d], k/v [T,K,d], cu_seqlens [B+1] int32; optional caches [B,K,S_max,d]."""
+    T, H, d = q.shape
+    K = k.shape[1]
+    B = cu_seqlens.shape[0] - 1
+    assert out.shape == q.shape and k.shape == (T, K, d) and v.shape == k.shape and cu_seqlens.dtype == torch.int32
+    S_max = k_cache.shape[2] if k_cache is not None else 0
+    if k_cache is not None:
+        assert k_cache.shape == (B, K, S_max, d) and v_cache is not None and v_cache.shape == k_cache.shape
+    _check("gqa_prefill_causal_varlen",
+           _lib.gqa_prefill_causal_varlen(_ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(cu_seqlens), B, T, H, K, S_max, d, float(scale), _dtype(q),
+                                          _stream(stream)))
 
 
 def gqa_meanpool_kv(dst, src, stream=None) -> None:

@@ -32,6 +32,7 @@ def test_header_declares_the_boundary():
                                          "gqa_decode_paged_workspace_bytes", "gqa_decode_paged",
                                          "gqa_decode_append_paged", "gqa_kv_append_paged",
                                          "gqa_decode_int8_workspace_bytes", "gqa_decode_int8", "gqa_kv_append_int8",
+                                         "gqa_prefill_causal_varlen",
                                          "gqa_prefill_causal",
                                          "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string"])
 
@@ -136,6 +137,18 @@ def test_int8_calls_reject_bad_arguments(lib):
     ws = lib.gqa_decode_int8_workspace_bytes
     assert ws(1, 8, 2, 64, 64, 0) == 0 and ws(1, 8, 2, 66, 128, 0) == 0
     assert ws(1, 64, 8, 131072, 128, 0) > 0
+
+
+def test_varlen_prefill_rejects_bad_arguments(lib):
+    f = lib.gqa_prefill_causal_varlen
+    # out, q, k, v, k_cache, v_cache, cu, B, T, H, K, S_max, d, scale, dtype, stream
+    assert f(P, P, P, P, None, None, P, 2, 100, 6, 4, 0, 128, 1.0, 1, None) == -2     # H % K != 0
+    assert f(P, P, P, P, None, None, P, 2, 100, 8, 4, 0, 96, 1.0, 1, None) == -2      # head dim
+    assert f(P, P, P, P, None, None, P, 2, 100, 8, 4, 0, 128, 1.0, 0, None) == -6     # f32
+    assert f(P, P, P, P, P, None, P, 2, 100, 8, 4, 64, 128, 1.0, 1, None) == -1       # one cache pointer
+    assert f(P, P, P, P, None, None, None, 2, 100, 8, 4, 0, 128, 1.0, 1, None) == -1  # no cu_seqlens
+    assert f(P, P + 8, P, P, None, None, P, 2, 100, 8, 4, 0, 128, 1.0, 1, None) == -3
+    assert f(None, None, None, None, None, None, None, 2, 0, 8, 4, 0, 128, 1.0, 1, None) == 0
 
 
 def test_prefill_rejects_bad_arguments(lib):
