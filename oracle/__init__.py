@@ -27,6 +27,11 @@ Page citations (title, section):
     head), value = code * scale; quantization in float32: scale = amax / 127,
     code = round-half-even(x / scale). Decoding an 8-bit cache is the decode
     of the values it holds.
+  * Fused K/V projection: "GQA 完全拆解", section 工程实现：权重布局、repeat 与
+    Kernel 融合 (GQA's W_K, W_V are [K, d_k, d_model]; inference engines merge
+    them into one W_KV [K, 2 d_k, d_model] so that one GEMM yields K and V).
+    The reading: W_KV[g] holds K's d_k rows, then V's; a token's K and V for
+    KV head g are W_KV[g] x, written to the cache at the token's key.
   * Varlen prefill: "GQA 完全拆解", section 主流模型里的 GQA：KV 缓存账本
     (continuous batching with the KV cache: requests of different lengths
     batched together); each sequence of a packed batch is prefilled causally
@@ -407,4 +412,36 @@ def prefill_cache_write_varlen(k, v, cu_seqlens, S_max: int, k_cache, v_cache):
         n = min(s1 - s0, S_max)
         kc[b, :, :n, :] = np.transpose(k[s0:s0 + n], (1, 0, 2))
         vc[b, :, :n, :] = np.transpose(v[s0:s0 + n], (1, 0, 2))
+    return kc, vc
+
+
+# ---------------------------------------------------------------------------
+# fused K/V projection into the cache (a matmul and row placement)
+
+def kv_project(x, w_kv) -> np.ndarray:
+    """x [..., d_model], w_kv [K, 2d, d_model] -> float64 [..., K, 2d]: W_KV[g] x for every KV head g
+    (the first d of the 2d outputs are K, the rest V)."""
+    xf = widen(np.asarray(x))
+    wf = widen(np.asarray(w_kv))
+    K, two_d, dm = wf.shape
+    out = xf.reshape(-1, dm) @ wf.reshape(K * two_d, dm).T  # a library matmul in float64
+    return out.reshape(*xf.shape[:-1], K, two_d)
+
+
+def kv_project_append(k_cache, v_cache, x, w_kv, pos, like_dtype=np.uint16):
+    """x [B, T, d_model], w_kv [K, 2d, d_model], pos [B] (or None: 0) -> copies of the caches [B, K, S_max, d]
+    with key pos[b] + i of every (b, g) set to the projection of token (b, i), rounded once to the
+    cache's type. A sequence whose rows would not fit (pos < 0 or pos + T > S_max) is left untouched."""
+    kc, vc = np.array(k_cache, copy=True), np.array(v_cache, copy=True)
+    B, T, _ = np.asarray(x).shape
+    K, two_d, _ = np.asarray(w_kv).shape
+    d = two_d // 2
+    S_max = kc.shape[2]
+    kv = round_to(kv_project(x, w_kv), like_dtype)  # [B, T, K, 2d]
+    for b in range(B):
+        p0 = 0 if pos is None else int(pos[b])
+        if p0 < 0 or p0 + T > S_max:
+            continue
+        kc[b, :, p0:p0 + T, :] = np.transpose(kv[b, :, :, :d], (1, 0, 2))
+        vc[b, :, p0:p0 + T, :] = np.transpose(kv[b, :, :, d:], (1, 0, 2))
     return kc, vc

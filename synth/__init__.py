@@ -346,3 +346,37 @@ def varlen_inputs(w: VarlenShape) -> dict:
     T = int(cu[-1])
     return {"lens": lens, "cu_seqlens": cu, "q": normal((T, w.H, w.d), BF16, w.seed, STREAM_Q),
             "k": normal((T, w.K, w.d), BF16, w.seed, STREAM_K), "v": normal((T, w.K, w.d), BF16, w.seed, STREAM_V)}
+
+
+# --------------------------------------------------------------------------
+# fused K/V projection: hidden states and a merged W_KV of the Llama-3-8B shape
+
+
+@dataclasses.dataclass(frozen=True)
+class ProjShape:
+    name: str
+    B: int
+    T: int        # new tokens per sequence (1: a decode step; the prompt length: a prefill)
+    K: int
+    d: int
+    d_model: int
+    S_max: int
+    seed: int
+
+
+PROJ_WORKLOADS = {
+    "kv_proj_decode_b8_t1_k8_d128_dm4096": ProjShape("kv_proj_decode_b8_t1_k8_d128_dm4096", 8, 1, 8, 128, 4096,
+                                                     8192, SEED_BASE + 6),
+    "kv_proj_prefill_b4_t4096_k8_d128_dm4096": ProjShape("kv_proj_prefill_b4_t4096_k8_d128_dm4096", 4, 4096, 8,
+                                                         128, 4096, 4096, SEED_BASE + 7),
+}
+
+
+def proj_inputs(w: ProjShape) -> dict:
+    """x [B, T, d_model] ~ N(0, 1), w_kv [K, 2d, d_model] ~ N(0, 1/d_model) (bf16), pos [B]: the key of each
+    sequence's first new token (decode: len - 1 of a full cache; prefill: 0)."""
+    x = normal((w.B, w.T, w.d_model), BF16, w.seed, STREAM_Q)
+    wf = normal((w.K, 2 * w.d, w.d_model), F32, w.seed, STREAM_K) / np.float32(np.sqrt(w.d_model))
+    wb = (wf.view(np.uint32) + 0x7FFF + ((wf.view(np.uint32) >> 16) & 1)) >> 16  # float32 -> bf16 bits, nearest even
+    pos = np.full(w.B, w.S_max - w.T, dtype=np.int32)
+    return {"x": x, "w_kv": wb.astype(np.uint16), "pos": pos}

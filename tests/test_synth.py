@@ -95,3 +95,11 @@ def test_int8_cache_codes_scales_and_padding():
     assert (c[~valid] == -128).all() and np.isnan(s[~valid]).all()
     c2, s2 = synth.int8_cache(4, 8, 16, 77, synth.STREAM_K8, synth.STREAM_KSCALE, lens, 2, lo=0.01, hi=0.02)
     assert np.array_equal(c, c2) and np.array_equal(s[valid], s2[valid])
+
+
+def test_projection_inputs():
+    w = synth.PROJ_WORKLOADS["kv_proj_decode_b8_t1_k8_d128_dm4096"]
+    inp = synth.proj_inputs(w)
+    assert inp["x"].shape == (8, 1, 4096) and inp["w_kv"].shape == (8, 256, 4096) and inp["w_kv"].dtype == np.uint16
+    wf = (inp["w_kv"].astype(np.uint32) << 16).view(np.float32)
+    assert abs(float(np.std(wf)) - 1 / 64) < 1e-3 and (inp["pos"] == 8191).all()
