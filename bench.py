@@ -293,6 +293,7 @@ PREFILL = "causal_prefill_b4_s4096_h32_k8_d128"
 PAGED_EXTRA = list(synth.PAGED_WORKLOADS)
 INT8_EXTRA = list(synth.INT8_WORKLOADS)
 VARLEN_EXTRA = list(synth.VARLEN_WORKLOADS)
+PROJ_EXTRA = list(synth.PROJ_WORKLOADS)
 
 
 class L2Flush:
@@ -364,6 +365,10 @@ def extra_measurements(args, only=None):
         if only is not None and name != only:
             continue
         res[name] = varlen_measurement(args, name, peaks, 20 if only is None else args.steps)
+    for name in PROJ_EXTRA:
+        if only is not None and name != only:
+            continue
+        res[name] = proj_measurement(args, name, peaks, 20 if only is None else args.steps)
     if only is not None and only != PREFILL:
         return res
     # causal prefill with the KV-cache write: FLOPs over the causal pairs (j <= i) only
@@ -537,6 +542,53 @@ def varlen_measurement(args, name, peaks, steps):
     return r
 
 
+def proj_measurement(args, name, peaks, steps):
+    """gqa_kv_project_append: a decode step is bound by streaming W_KV (GB/s of weights and activations),
+    a prompt by the tensor cores (TFLOP/s)."""
+    import torch
+
+    from kv_cache_02_b200 import gqa
+
+    w = synth.PROJ_WORKLOADS[name]
+    inp = synth.proj_inputs(w)
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).cuda()
+
+    x, wk, pos = to_dev(inp["x"]), to_dev(inp["w_kv"]), to_dev(inp["pos"])
+    kc = torch.zeros((w.B, w.K, w.S_max, w.d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    wsb = gqa.gqa_kv_project_workspace_bytes(w.B, w.T, w.K, w.d, w.d_model)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
+    times = []
+    for it in range(args.warmup + steps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        gqa.gqa_kv_project_append(kc, vc, x, wk, pos, ws)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            times.append(a.elapsed_time(b))
+    if gqa.gqa_get_last_error() != (0, 0):
+        raise RuntimeError(f"device error in {name}")
+    ms = statistics.median(times)
+    M, N = w.B * w.T, w.K * 2 * w.d
+    flops = 2.0 * M * N * w.d_model
+    byts = (N * w.d_model + M * w.d_model + M * N) * 2  # W, x read once; the K/V rows written
+    r = {"ms": round(ms, 5), "flops": flops, "bytes": byts, "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1),
+         "GB/s": round(byts / (ms * 1e-3) / 1e9, 1), "l2": "flushed (512 MiB write, then 512 MiB read)"}
+    if M < 512:
+        r["frac_of_measured_hbm"] = round(r["GB/s"] / peaks["hbm_gbs"], 4)
+    else:
+        r["frac_of_measured_bf16_burst"] = round(r["TFLOP/s"] / peaks["bf16_tflops"], 4)
+    del x, wk, pos, kc, vc, ws, flush
+    torch.cuda.empty_cache()
+    return r
+
+
 def cpu_baseline(inp, scale, kv_bytes_layer):
     """The oracle as it stands, on all host cores, over one full layer of the workload."""
     import oracle
@@ -591,7 +643,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads and the CPU baseline")
-    ap.add_argument("--only", choices=DECODE_EXTRA + PAGED_EXTRA + INT8_EXTRA + VARLEN_EXTRA + [PREFILL],
+    ap.add_argument("--only", choices=DECODE_EXTRA + PAGED_EXTRA + INT8_EXTRA + VARLEN_EXTRA + PROJ_EXTRA + [PREFILL],
                     default=None,
                     help="time one other workload alone (for profiling); prints its own JSON, not the contract line")
     ap.add_argument("--layers", type=int, default=32,

@@ -308,6 +308,36 @@ GQA_API int gqa_prefill_causal_varlen(void* out, const void* q, const void* k, c
                                       int S_max, int d, float scale, gqa_dtype dtype, gqa_stream_t stream);
 
 /*
+ * gqa_kv_project_append - the K/V projection of new tokens, written straight
+ * into the cache.
+ *
+ * "GQA 完全拆解", section 工程实现：权重布局、repeat 与 Kernel 融合: GQA's W_K and
+ * W_V are [K, d_k, d_model]; inference engines merge them into one
+ * W_KV [K, 2 d_k, d_model] so that one GEMM yields K and V. Here:
+ *
+ *   k_cache[b, g, pos[b] + i, :] = (W_KV[g] x[b, i, :])[0 : d]
+ *   v_cache[b, g, pos[b] + i, :] = (W_KV[g] x[b, i, :])[d : 2d]
+ *
+ * x         : [B, T, d_model] bfloat16: T new tokens per sequence (1 for a
+ *             decode step, the prompt for a prefill).
+ * w_kv      : [K, 2d, d_model] bfloat16: K's d rows, then V's, per KV head.
+ * pos       : [B] int32, device: the key of each sequence's first new token,
+ *             or NULL (0 for every sequence). pos[b] < 0 or pos[b] + T >
+ *             S_max sets GQA_DEVERR_APPEND_POS and leaves that sequence's
+ *             rows unwritten.
+ * k_cache,
+ * v_cache   : [B, K, S_max, d] bfloat16, written in place (only those rows).
+ * workspace : gqa_kv_project_workspace_bytes(...) bytes of device scratch
+ *             (0 when the GEMM needs no split of d_model); no initialisation.
+ * d is 64 or 128 and d_model a multiple of 64; fp32 accumulation, one
+ * rounding to bf16; GQA_BF16 only.
+ */
+GQA_API size_t gqa_kv_project_workspace_bytes(int B, int T, int K, int d, int d_model);
+GQA_API int gqa_kv_project_append(void* k_cache, void* v_cache, const void* x, const void* w_kv, const int32_t* pos,
+                                  int B, int T, int K, int S_max, int d, int d_model, void* workspace,
+                                  size_t workspace_bytes, gqa_dtype dtype, gqa_stream_t stream);
+
+/*
  * gqa_meanpool_kv - MHA -> GQA conversion by mean pooling of heads.
  *
  * "分組查詢注意力", section 模型轉換與 Uptraining, and "GQA 完全拆解", section

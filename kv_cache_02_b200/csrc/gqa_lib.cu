@@ -21,6 +21,7 @@
 #include "decode.cuh"
 #include "decode_wide.cuh"
 #include "prefill.cuh"
+#include "kv_proj.cuh"
 
 namespace {
 
@@ -385,6 +386,55 @@ int launch_prefill_varlen(void* out, const void* q, const void* k, const void* v
   return launch_status();
 }
 
+// Fused K/V projection: d_model is split over CTAs (powers of two, at least
+// 4 pipeline steps each) while the token tiles x heads leave SMs idle.
+struct ProjPlan {
+  int splits = 1;
+  long long grid = 0;
+  size_t ws_bytes = 0;
+};
+
+ProjPlan plan_proj(long long M, int K, int d, int d_model, int sms) {
+  ProjPlan pl;
+  const int ksteps = d_model / gqa::kPjBK;
+  const long long base = (M + gqa::kPjBM - 1) / gqa::kPjBM * K;
+  while (base * pl.splits < sms && ksteps % (pl.splits * 2) == 0 && ksteps / (pl.splits * 2) >= 4) pl.splits *= 2;
+  pl.grid = base * pl.splits;
+  pl.ws_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)M * K * 2 * d * sizeof(float) : 0;
+  return pl;
+}
+
+bool valid_proj(int B, int T, int K, int S_max, int d, int d_model) {
+  if (B < 0 || T <= 0 || K <= 0 || S_max <= 0 || d_model <= 0) return false;
+  if ((d != 64 && d != 128) || d_model % gqa::kPjBK != 0) return false;
+  if ((long long)B * T >= (1ll << 31) || (long long)K * 2 * d >= (1ll << 31)) return false;
+  return true;
+}
+
+template <int D>
+int launch_proj_d(const ProjPlan& pl, gqa::ProjParams p, const void* x, const void* w, int d_model, cudaStream_t st,
+                  int sms) {
+  using C = gqa::PjCfg<D>;
+  CUtensorMap tx, tw;
+  if (!encode_rows_bf16(&tx, x, (uint64_t)p.M, (uint64_t)d_model, gqa::kPjBM) ||
+      !encode_rows_bf16(&tw, w, (uint64_t)p.K * C::kN, (uint64_t)d_model, C::kN))
+    return GQA_ERR_CUDA;
+  static bool configured[kMaxDevices] = {false};
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
+    if (cudaFuncSetAttribute(gqa::kv_proj_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+      return GQA_ERR_CUDA;
+    configured[dev] = true;
+  }
+  gqa::kv_proj_kernel<D><<<(unsigned)pl.grid, gqa::kPjThreads, C::kSmemBytes, st>>>(tx, tw, p);
+  if (pl.splits > 1) {
+    const long long work = (long long)p.M * p.K * (C::kN / 8);
+    gqa::kv_proj_finalize_kernel<D><<<grid_for(work, 256, sms), 256, 0, st>>>(p);
+  }
+  return launch_status();
+}
+
 }  // namespace
 
 // ============================================================================
@@ -670,6 +720,42 @@ int gqa_kv_append_int8(int8_t* k_codes, float* k_scales, int8_t* v_codes, float*
       k_codes, k_scales, v_codes, v_scales, static_cast<const __nv_bfloat16*>(k_new),
       static_cast<const __nv_bfloat16*>(v_new), pos, B, K, S_max);
   return launch_status();
+}
+
+size_t gqa_kv_project_workspace_bytes(int B, int T, int K, int d, int d_model) {
+  if (!valid_proj(B, T, K, 1, d, d_model)) return 0;
+  return plan_proj((long long)B * T, K, d, d_model, sm_count(current_device())).ws_bytes;
+}
+
+int gqa_kv_project_append(void* k_cache, void* v_cache, const void* x, const void* w_kv, const int32_t* pos, int B,
+                          int T, int K, int S_max, int d, int d_model, void* workspace, size_t workspace_bytes,
+                          gqa_dtype dtype, gqa_stream_t stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (B < 0 || T <= 0 || K <= 0 || S_max <= 0 || d_model <= 0) return GQA_ERR_INVALID_ARG;
+  if (!valid_proj(B, T, K, S_max, d, d_model)) return GQA_ERR_SHAPE;
+  if (dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
+  if (B == 0) return GQA_OK;
+  if (!k_cache || !v_cache || !x || !w_kv) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(x) || !aligned16(w_kv)) return GQA_ERR_ALIGN;
+  const int sms = sm_count(current_device());
+  const ProjPlan pl = plan_proj((long long)B * T, K, d, d_model, sms);
+  if (pl.ws_bytes > 0 && (!workspace || workspace_bytes < pl.ws_bytes)) return GQA_ERR_INVALID_ARG;
+  if (pl.ws_bytes > 0 && !aligned16(workspace)) return GQA_ERR_ALIGN;
+  gqa::ProjParams p;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.pos = pos;
+  p.ws = static_cast<float*>(workspace);
+  p.B = B;
+  p.T = T;
+  p.K = K;
+  p.S_max = S_max;
+  p.M = B * T;
+  p.splits = pl.splits;
+  p.ksteps_per_split = d_model / gqa::kPjBK / pl.splits;
+  cudaStream_t st = (cudaStream_t)stream;
+  return d == 128 ? launch_proj_d<128>(pl, p, x, w_kv, d_model, st, sms)
+                  : launch_proj_d<64>(pl, p, x, w_kv, d_model, st, sms);
 }
 
 size_t gqa_decode_paged_workspace_bytes(int B, int H, int K, int d, int block_size, int max_blocks, int num_splits) {

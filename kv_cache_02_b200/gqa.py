@@ -30,6 +30,7 @@ GQA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 EXPORTED = ("gqa_kv_append", "gqa_decode_workspace_bytes", "gqa_decode", "gqa_decode_append", "gqa_decode_noalloc",
             "gqa_decode_paged_workspace_bytes", "gqa_decode_paged", "gqa_decode_append_paged", "gqa_kv_append_paged",
             "gqa_decode_int8_workspace_bytes", "gqa_decode_int8", "gqa_kv_append_int8", "gqa_prefill_causal_varlen",
+            "gqa_kv_project_workspace_bytes", "gqa_kv_project_append",
             "gqa_prefill_causal", "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string")
 
 
@@ -73,6 +74,10 @@ def _load():
     lib.gqa_prefill_causal.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gqa_prefill_causal_varlen.restype = I
     lib.gqa_prefill_causal_varlen.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.gqa_kv_project_workspace_bytes.restype = SZ
+    lib.gqa_kv_project_workspace_bytes.argtypes = [I, I, I, I, I]
+    lib.gqa_kv_project_append.restype = I
+    lib.gqa_kv_project_append.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, SZ, I, P]
     lib.gqa_meanpool_kv.restype = I
     lib.gqa_meanpool_kv.argtypes = [P, P, I64, I, I, I64, I, P]
     lib.gqa_get_last_error.restype = I
@@ -284,6 +289,25 @@ def gqa_prefill_causal_varlen(out, q, k, v, cu_seqlens, scale: float, k_cache=No
            _lib.gqa_prefill_causal_varlen(_ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
                                           _ptr(cu_seqlens), B, T, H, K, S_max, d, float(scale), _dtype(q),
                                           _stream(stream)))
+
+
+def gqa_kv_project_workspace_bytes(B: int, T: int, K: int, d: int, d_model: int) -> int:
+    return int(_lib.gqa_kv_project_workspace_bytes(B, T, K, d, d_model))
+
+
+def gqa_kv_project_append(k_cache, v_cache, x, w_kv, pos=None, workspace=None, stream=None) -> None:
+    """x [B,T,d_model], w_kv [K,2d,d_model] (bf16); caches [B,K,S_max,d]; pos [B] int32 or None (0)."""
+    B, T, d_model = x.shape
+    K, two_d, dm = w_kv.shape
+    d = two_d // 2
+    S_max = k_cache.shape[2]
+    assert dm == d_model and k_cache.shape == (B, K, S_max, d) and v_cache.shape == k_cache.shape
+    if pos is not None:
+        assert pos.dtype == torch.int32 and pos.shape == (B,)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("gqa_kv_project_append",
+           _lib.gqa_kv_project_append(_ptr(k_cache), _ptr(v_cache), _ptr(x), _ptr(w_kv), _ptr(pos), B, T, K, S_max,
+                                      d, d_model, _ptr(workspace), ws_bytes, _dtype(x), _stream(stream)))
 
 
 def gqa_meanpool_kv(dst, src, stream=None) -> None:

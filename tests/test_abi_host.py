@@ -32,7 +32,8 @@ def test_header_declares_the_boundary():
                                          "gqa_decode_paged_workspace_bytes", "gqa_decode_paged",
                                          "gqa_decode_append_paged", "gqa_kv_append_paged",
                                          "gqa_decode_int8_workspace_bytes", "gqa_decode_int8", "gqa_kv_append_int8",
-                                         "gqa_prefill_causal_varlen",
+                                         "gqa_prefill_causal_varlen", "gqa_kv_project_workspace_bytes",
+                                         "gqa_kv_project_append",
                                          "gqa_prefill_causal",
                                          "gqa_meanpool_kv", "gqa_get_last_error", "gqa_status_string"])
 
@@ -149,6 +150,19 @@ def test_varlen_prefill_rejects_bad_arguments(lib):
     assert f(P, P, P, P, None, None, None, 2, 100, 8, 4, 0, 128, 1.0, 1, None) == -1  # no cu_seqlens
     assert f(P, P + 8, P, P, None, None, P, 2, 100, 8, 4, 0, 128, 1.0, 1, None) == -3
     assert f(None, None, None, None, None, None, None, 2, 0, 8, 4, 0, 128, 1.0, 1, None) == 0
+
+
+def test_projection_rejects_bad_arguments(lib):
+    f = lib.gqa_kv_project_append
+    # k_cache, v_cache, x, w, pos, B, T, K, S_max, d, d_model, ws, ws_bytes, dtype, stream
+    assert f(P, P, P, P, None, 2, 1, 8, 64, 96, 4096, None, 0, 1, None) == -2    # head dim
+    assert f(P, P, P, P, None, 2, 1, 8, 64, 128, 4000, None, 0, 1, None) == -2   # d_model not a multiple of 64
+    assert f(P, P, P, P, None, 2, 1, 8, 64, 128, 4096, None, 0, 0, None) == -6   # f32
+    assert f(P, P, P, P, None, 2, 1, 8, 64, 128, 4096, None, 0, 1, None) == -1   # needs a workspace (8 tokens)
+    assert f(P, P, P + 2, P, None, 2, 1, 8, 64, 128, 4096, None, 0, 1, None) == -3
+    assert f(None, None, None, None, None, 0, 1, 8, 64, 128, 4096, None, 0, 1, None) == 0
+    ws = lib.gqa_kv_project_workspace_bytes
+    assert ws(8, 1, 8, 128, 4096) > 0 and ws(4, 4096, 8, 128, 4096) == 0 and ws(8, 1, 8, 128, 100) == 0
 
 
 def test_prefill_rejects_bad_arguments(lib):
