@@ -389,16 +389,23 @@ int launch_prefill_varlen(void* out, const void* q, const void* k, const void* v
 // Fused K/V projection: d_model is split over CTAs (powers of two, at least
 // 4 pipeline steps each) while the token tiles x heads leave SMs idle.
 struct ProjPlan {
+  bool small = false;
   int splits = 1;
   long long grid = 0;
   size_t ws_bytes = 0;
 };
 
+// small: at most 16 tokens, the operand-swapped kernel (W_KV rows as M);
+// it fits three CTAs per SM, so it aims at two per SM.
 ProjPlan plan_proj(long long M, int K, int d, int d_model, int sms) {
   ProjPlan pl;
   const int ksteps = d_model / gqa::kPjBK;
-  const long long base = (M + gqa::kPjBM - 1) / gqa::kPjBM * K;
-  while (base * pl.splits < sms && ksteps % (pl.splits * 2) == 0 && ksteps / (pl.splits * 2) >= 4) pl.splits *= 2;
+  pl.small = M <= gqa::kPsTok;
+  const long long base = pl.small ? (long long)K * 2 * d / gqa::kPsRows : (M + gqa::kPjBM - 1) / gqa::kPjBM * K;
+  const long long target = pl.small ? 2ll * sms : sms;
+  while (base * pl.splits < target && ksteps % (pl.splits * 2) == 0 && ksteps / (pl.splits * 2) >= 4 &&
+         pl.splits * 2 <= gqa::kPjMaxSplits)
+    pl.splits *= 2;
   pl.grid = base * pl.splits;
   pl.ws_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)M * K * 2 * d * sizeof(float) : 0;
   return pl;
@@ -423,14 +430,36 @@ int launch_proj_d(const ProjPlan& pl, gqa::ProjParams p, const void* x, const vo
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
     if (cudaFuncSetAttribute(gqa::kv_proj_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(gqa::kv_proj_small_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gqa::PsCfg::kSmemBytes) != cudaSuccess)
       return GQA_ERR_CUDA;
     configured[dev] = true;
   }
-  gqa::kv_proj_kernel<D><<<(unsigned)pl.grid, gqa::kPjThreads, C::kSmemBytes, st>>>(tx, tw, p);
-  if (pl.splits > 1) {
-    const long long work = (long long)p.M * p.K * (C::kN / 8);
-    gqa::kv_proj_finalize_kernel<D><<<grid_for(work, 256, sms), 256, 0, st>>>(p);
+  if (pl.small) {
+    CUtensorMap tx16, tw128;
+    if (!encode_rows_bf16(&tx16, x, (uint64_t)p.M, (uint64_t)d_model, gqa::kPsTok) ||
+        !encode_rows_bf16(&tw128, w, (uint64_t)p.K * C::kN, (uint64_t)d_model, gqa::kPsRows))
+      return GQA_ERR_CUDA;
+    gqa::kv_proj_small_kernel<D><<<(unsigned)pl.grid, gqa::kPjThreads, gqa::PsCfg::kSmemBytes, st>>>(tx16, tw128, p);
+  } else {
+    gqa::kv_proj_kernel<D><<<(unsigned)pl.grid, gqa::kPjThreads, C::kSmemBytes, st>>>(tx, tw, p);
+  }
+  if (pl.splits > 1) {  // as a programmatic dependent launch: its launch overlaps the GEMM
+    const long long work = (long long)p.M * p.K * C::kN;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid_for(work, 256, sms));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gqa::kv_proj_finalize_kernel<D>, p) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ERR_CUDA;
+    }
   }
   return launch_status();
 }

@@ -13,10 +13,11 @@
 // fp32 accumulator in TMEM (lane = token row). Warp roles: 0-3 epilogue,
 // 4 TMA producer, 5 TMEM allocation and the MMA-issuing thread.
 //
-// When the token tiles and heads alone would leave SMs idle (a decode step
-// has 8 tokens: 8 CTAs), d_model is split over CTAs: each split writes its
-// fp32 partial tile to a workspace slice of its own (no atomics, nothing to
-// zero) and kv_proj_finalize_kernel sums the splits and writes the rows.
+// When the token tiles and heads alone would leave SMs idle, d_model is
+// split over CTAs: each split writes its fp32 partial tile to a workspace
+// slice of its own (no atomics, nothing to zero) and kv_proj_finalize_kernel
+// sums the splits and writes the rows. A decode step (a few tokens) uses
+// kv_proj_small_kernel, with the operands swapped.
 #pragma once
 
 #include "common.cuh"
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the finalize pass may be scheduled
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -185,38 +187,164 @@ __global__ void __launch_bounds__(kPjThreads, 1)
   }
 }
 
+// A decode step (at most kPsTok tokens): the operands swap. A = 128 rows of
+// W_KV (outputs), B = the tokens (padded to 16), D = [128 outputs x 16
+// tokens] in TMEM (lane = output), so the MMA does 16x less padding work
+// than with tokens as M and every CTA streams its own slice of W_KV.
+// Epilogue thread r holds output r for every token: across a warp 32
+// consecutive outputs of one token, 64 contiguous bytes of a cache row.
+constexpr int kPsRows = 128;  // W_KV rows (outputs) per CTA
+constexpr int kPsTok = 16;    // tokens (MMA N)
+
+struct PsCfg {
+  static constexpr int kABytes = kPsRows * kPjBK * 2;  // 16 KB of W
+  static constexpr int kBBytes = kPsTok * kPjBK * 2;   // 2 KB of x
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOff = kPjStages * kStageBytes;
+  static constexpr int kNumBars = 2 * kPjStages + 1;
+  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
+  static constexpr int kTmemCols = 32;  // 16 used (the allocation minimum is 32)
+};
+
+template <int D>
+__global__ void __launch_bounds__(kPjThreads)
+    kv_proj_small_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                         const ProjParams p) {
+  using C = PsCfg;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kPjStages;
+  uint64_t* acc_full = empty + kPjStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) raise_error(GQA_DEVERR_TIMEOUT);
+    return;
+  }
+  const int ft = (int)(blockIdx.x / p.splits);  // tile of 128 W_KV rows
+  const int sp = (int)(blockIdx.x % p.splits);
+  const int k_begin = sp * p.ksteps_per_split;
+  const int nk = p.ksteps_per_split;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPjStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the finalize pass may be scheduled
+
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tensormap(&tm_x);
+      prefetch_tensormap(&tm_w);
+      const uint64_t pol_x = l2_policy_evict_last();
+      const uint64_t pol_w = l2_policy_evict_first();
+      int issued = 0;
+      for (int j = 0; j < nk; ++j) {
+        const int s = j % kPjStages;
+        if (j >= kPjStages && !mbar_wait_bounded(&empty[s], ((j / kPjStages) - 1) & 1)) break;
+        uint8_t* st = smem + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)C::kStageBytes);
+        const int kx = (k_begin + j) * kPjBK;
+        tma_load_2d(st, &tm_w, kx, ft * kPsRows, &full[s], pol_w);
+        tma_load_2d(st + C::kABytes, &tm_x, kx, 0, &full[s], pol_x);
+        ++issued;
+      }
+      for (int j = max(0, issued - kPjStages); j < issued; ++j) mbar_wait_bounded(&full[j % kPjStages], (j / kPjStages) & 1);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kPsRows, kPsTok, false, false);
+      bool ok = true;
+      for (int j = 0; j < nk && ok; ++j) {
+        const int s = j % kPjStages;
+        if (!(ok = mbar_wait_bounded(&full[s], (j / kPjStages) & 1))) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + s * C::kStageBytes);
+        const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+        for (int kk = 0; kk < kPjBK / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+          tc_mma(tmem, ad, bd, idesc, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+      }
+      tc_commit(acc_full);
+    }
+  } else {
+    const int f = ft * kPsRows + threadIdx.x;  // W_KV row: head f / 2D, K (< D) or V, dim f % D
+    const int g = f / (2 * D), jd = f % (2 * D);
+    if (__all_sync(0xffffffffu, mbar_wait_bounded(acc_full, 0))) {
+      tc_fence_after();
+      float o[16];
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), o);
+      tc_wait_ld();
+      const size_t ncols = (size_t)p.K * 2 * D;
+#pragma unroll
+      for (int t = 0; t < kPsTok; ++t) {
+        if (t >= p.M) break;
+        if (p.splits > 1) {
+          p.ws[((size_t)sp * p.M + t) * ncols + f] = o[t];
+        } else {
+          size_t row = 0;
+          if (!proj_row(p, t, g, row)) continue;
+          __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(jd < D ? p.k_cache : p.v_cache);
+          cache[row * D + (jd % D)] = __float2bfloat16_rn(o[t]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
 // Split d_model: the sum of the splits' partials, rounded once to bf16 and
-// written at the token's key. One thread per 8 outputs of a (token, head).
+// written at the token's key. One thread per output (consecutive outputs in
+// consecutive threads); the splits' partials (at most kPjMaxSplits) are all
+// loaded before any is summed, one round trip. Launched as a programmatic
+// dependent of the GEMM: it waits for that grid before reading.
+constexpr int kPjMaxSplits = 16;
+
 template <int D>
 __global__ void kv_proj_finalize_kernel(const ProjParams p) {
   constexpr int kN = 2 * D;
-  const long long total = (long long)p.M * p.K * (kN / 8);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const size_t ncols = (size_t)p.K * kN;
+  const long long total = (long long)p.M * (long long)ncols;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
-    const int c8 = (int)(i % (kN / 8));
-    const long long mg = i / (kN / 8);
-    const int g = (int)(mg % p.K), m = (int)(mg / p.K);
+    const int f = (int)(i % (long long)ncols);
+    const int m = (int)(i / (long long)ncols);
+    const int g = f / kN, j = f % kN;
     size_t row = 0;
     if (!proj_row(p, m, g, row)) continue;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < p.splits; ++s) {
-      const float4* src = reinterpret_cast<const float4*>(p.ws + ((size_t)s * p.M + m) * ((size_t)p.K * kN) +
-                                                          (size_t)g * kN + c8 * 8);
-      const float4 a = __ldcg(src), b = __ldcg(src + 1);
-      acc[0] += a.x;
-      acc[1] += a.y;
-      acc[2] += a.z;
-      acc[3] += a.w;
-      acc[4] += b.x;
-      acc[5] += b.y;
-      acc[6] += b.z;
-      acc[7] += b.w;
-    }
-    const int c = c8 * 8;
-    __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(c < D ? p.k_cache : p.v_cache);
-    *reinterpret_cast<uint4*>(cache + row * D + (c % D)) =
-        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                   pack_bf16x2(acc[6], acc[7]));
+    float v[kPjMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kPjMaxSplits; ++s)
+      v[s] = s < p.splits ? __ldcg(p.ws + ((size_t)s * p.M + m) * ncols + f) : 0.f;
+    float acc = 0.f;
+#pragma unroll
+    for (int s = 0; s < kPjMaxSplits; ++s) acc += v[s];
+    __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(j < D ? p.k_cache : p.v_cache);
+    cache[row * D + (j % D)] = __float2bfloat16_rn(acc);
   }
 }
 
