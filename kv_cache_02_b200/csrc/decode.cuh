@@ -599,8 +599,8 @@ __device__ __forceinline__ ItemCoord item_coord_n(const DecodeParams& p, int ite
   ItemCoord c;
   c.hsl = item % p.hslices;
   const int rest = item / p.hslices;
-  c.split = rest % p.nsplit;
-  c.unit = rest / p.nsplit;
+  c.unit = rest % (p.B * p.K);  // split-major: the short last splits of the units come last
+  c.split = rest / (p.B * p.K);
   c.b = c.unit / p.K;
   c.g = c.unit % p.K;
   c.h0 = c.g * p.G + c.hsl * heads_per_cta;
@@ -612,8 +612,8 @@ __device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item)
   ItemCoord c;
   c.hsl = item % p.hslices;
   const int rest = item / p.hslices;
-  c.split = rest % p.nsplit;
-  c.unit = rest / p.nsplit;
+  c.unit = rest % (p.B * p.K);  // split-major: the short last splits of the units come last
+  c.split = rest / (p.B * p.K);
   c.b = c.unit / p.K;
   c.g = c.unit % p.K;
   c.h0 = c.g * p.G + c.hsl * kDecHeadsPerCta;
