@@ -412,6 +412,9 @@ __device__ __forceinline__ void warp_tile(WarpState<D>& st, const uint32_t (&qf)
 // 16-dim step d0 being dim d0 + i8_dim(m) (see stash_warp_state).
 __device__ __forceinline__ int i8_dim(int m) { return 4 * ((m & 7) >> 1) + (m & 1) + ((m >> 3) << 1); }
 
+// One warp's 32 keys (kb .. kb+31) of the 8-bit tile in `stage`, as two
+// independent 16-key blocks (a: kb.., b: kb+16..) so that two MMA chains are
+// in flight; `rows` keys of the tile are valid, kb < rows.
 template <int D>
 __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&qf)[D / 16][2], uint32_t stage_addr,
                                              const float* sk, const float* sv, int kb, int rows, int lane,
@@ -423,30 +426,41 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
   const int row = kb + (lane & 7) + ((lane >> 3) & 1) * 8;
   const int ch = lane >> 4;
 
-  // S^T = K * Q^T, two 16-dim steps per ldmatrix
-  float c[4] = {0.f, 0.f, 0.f, 0.f};
+  // S^T = K * Q^T for both blocks, two 16-dim steps per ldmatrix
+  float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int j = 0; j < D / 32; ++j) {
-    uint32_t r0, r1, r2, r3;
-    ldmatrix_x4(k_base + sw128(row, 2 * j + ch), r0, r1, r2, r3);
-    uint32_t l0, h0, l1, h1, l2, h2, l3, h3;
-    int8x4_to_f16x2(r0, l0, h0);
-    int8x4_to_f16x2(r1, l1, h1);
-    int8x4_to_f16x2(r2, l2, h2);
-    int8x4_to_f16x2(r3, l3, h3);
-    mma_f16_16816(c, l0, l1, h0, h1, qf[2 * j][0], qf[2 * j][1]);
-    mma_f16_16816(c, l2, l3, h2, h3, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+    uint32_t r[4], t[4];
+    ldmatrix_x4(k_base + sw128(row, 2 * j + ch), r[0], r[1], r[2], r[3]);
+    ldmatrix_x4(k_base + sw128(row + 16, 2 * j + ch), t[0], t[1], t[2], t[3]);
+    uint32_t rl[4], rh[4], tl[4], th[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int8x4_to_f16x2(r[i], rl[i], rh[i]);
+      int8x4_to_f16x2(t[i], tl[i], th[i]);
+    }
+    mma_f16_16816(ca, rl[0], rl[1], rh[0], rh[1], qf[2 * j][0], qf[2 * j][1]);
+    mma_f16_16816(cb, tl[0], tl[1], th[0], th[1], qf[2 * j][0], qf[2 * j][1]);
+    mma_f16_16816(ca, rl[2], rl[3], rh[2], rh[3], qf[2 * j + 1][0], qf[2 * j + 1][1]);
+    mma_f16_16816(cb, tl[2], tl[3], th[2], th[3], qf[2 * j + 1][0], qf[2 * j + 1][1]);
   }
 
-  // online softmax (key kb + lane/4 in c0/c1, +8 in c2/c3), scores scaled by the key's K scale
+  // online softmax over the 32 keys: key kb + lane/4 + 8 i for i = 0..3
+  // (block a: c0/c1 and c2/c3, block b: the same, 16 keys on), each score
+  // scaled by its key's K scale
   const int key0 = kb + (lane >> 2);
-  const bool v0 = key0 < rows, v1 = key0 + 8 < rows;
-  const float s0 = v0 ? sk[key0] * scale_log2 : 0.f, s1 = v1 ? sk[key0 + 8] * scale_log2 : 0.f;
-  const float x0 = v0 ? c[0] * s0 : -INFINITY;
-  const float x1 = v0 ? c[1] * s0 : -INFINITY;
-  const float x2 = v1 ? c[2] * s1 : -INFINITY;
-  const float x3 = v1 ? c[3] * s1 : -INFINITY;
-  float mx_a = fmaxf(x0, x2), mx_b = fmaxf(x1, x3);
+  bool vk[4];
+  float xa[4], xb[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    vk[i] = key0 + 8 * i < rows;
+    const float sc = vk[i] ? sk[key0 + 8 * i] * scale_log2 : 0.f;
+    const float* c = i < 2 ? ca : cb;
+    xa[i] = vk[i] ? c[2 * (i & 1)] * sc : -INFINITY;
+    xb[i] = vk[i] ? c[2 * (i & 1) + 1] * sc : -INFINITY;
+  }
+  float mx_a = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
+  float mx_b = fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3]));
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
@@ -456,10 +470,14 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
   const float al_a = fast_exp2(st.m_a - mn_a), al_b = fast_exp2(st.m_b - mn_b);
   st.m_a = mn_a;
   st.m_b = mn_b;
-  const float p0 = fast_exp2(x0 - mn_a), p1 = fast_exp2(x1 - mn_b);
-  const float p2 = fast_exp2(x2 - mn_a), p3 = fast_exp2(x3 - mn_b);
-  st.l_a = st.l_a * al_a + p0 + p2;
-  st.l_b = st.l_b * al_b + p1 + p3;
+  float pa[4], pb[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    pa[i] = fast_exp2(xa[i] - mn_a);
+    pb[i] = fast_exp2(xb[i] - mn_b);
+  }
+  st.l_a = st.l_a * al_a + ((pa[0] + pa[1]) + (pa[2] + pa[3]));
+  st.l_b = st.l_b * al_b + ((pb[0] + pb[1]) + (pb[2] + pb[3]));
 #pragma unroll
   for (int md = 0; md < D / 16; ++md) {
     st.o[md][0] *= al_a;
@@ -469,24 +487,33 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
   }
 
   // P^T times the V scales (keys past the valid rows: 0, their scales are never read)
-  const float w0 = v0 ? sv[key0] : 0.f, w1 = v1 ? sv[key0 + 8] : 0.f;
-  const uint32_t pb0 = movmatrix_trans(pack_f16x2(p0 * w0, p1 * w0));
-  const uint32_t pb1 = movmatrix_trans(pack_f16x2(p2 * w1, p3 * w1));
+  uint32_t pt[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float w = vk[i] ? sv[key0 + 8 * i] : 0.f;
+    pt[i] = movmatrix_trans(pack_f16x2(pa[i] * w, pb[i] * w));
+  }
 
-  // O^T += V^T * P^T, two 16-dim steps per ldmatrix
+  // O^T += V^T * P^T for both blocks, two 16-dim steps per ldmatrix
 #pragma unroll
   for (int j = 0; j < D / 32; ++j) {
-    uint32_t r0, r1, r2, r3;
-    ldmatrix_x4(v_base + sw128(row, 2 * j + ch), r0, r1, r2, r3);
-    uint32_t l0, h0, l1, h1, l2, h2, l3, h3;
-    int8x4_to_f16x2(r0, l0, h0);
-    int8x4_to_f16x2(r1, l1, h1);
-    int8x4_to_f16x2(r2, l2, h2);
-    int8x4_to_f16x2(r3, l3, h3);
-    mma_f16_16816(st.o[2 * j], movmatrix_trans(l0), movmatrix_trans(h0), movmatrix_trans(l1), movmatrix_trans(h1),
-                  pb0, pb1);
-    mma_f16_16816(st.o[2 * j + 1], movmatrix_trans(l2), movmatrix_trans(h2), movmatrix_trans(l3),
-                  movmatrix_trans(h3), pb0, pb1);
+    uint32_t r[4], t[4];
+    ldmatrix_x4(v_base + sw128(row, 2 * j + ch), r[0], r[1], r[2], r[3]);
+    ldmatrix_x4(v_base + sw128(row + 16, 2 * j + ch), t[0], t[1], t[2], t[3]);
+    uint32_t rl[4], rh[4], tl[4], th[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int8x4_to_f16x2(r[i], rl[i], rh[i]);
+      int8x4_to_f16x2(t[i], tl[i], th[i]);
+    }
+    mma_f16_16816(st.o[2 * j], movmatrix_trans(rl[0]), movmatrix_trans(rh[0]), movmatrix_trans(rl[1]),
+                  movmatrix_trans(rh[1]), pt[0], pt[1]);
+    mma_f16_16816(st.o[2 * j + 1], movmatrix_trans(rl[2]), movmatrix_trans(rh[2]), movmatrix_trans(rl[3]),
+                  movmatrix_trans(rh[3]), pt[0], pt[1]);
+    mma_f16_16816(st.o[2 * j], movmatrix_trans(tl[0]), movmatrix_trans(th[0]), movmatrix_trans(tl[1]),
+                  movmatrix_trans(th[1]), pt[2], pt[3]);
+    mma_f16_16816(st.o[2 * j + 1], movmatrix_trans(tl[2]), movmatrix_trans(th[2]), movmatrix_trans(tl[3]),
+                  movmatrix_trans(th[3]), pt[2], pt[3]);
   }
 }
 
@@ -814,14 +841,17 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       if (si.new_row >= 0 && (si.new_row >> 4) == warp)
         append_row<D, kPaged>(p, cur, smem + s * C::kStageBytes, si.new_row, lane);
     }
-    if (kb < si.rows) {
-      if constexpr (kInt8) {
+    if constexpr (kInt8) {
+      // warps 0-1 take the even tiles of the ring, warps 2-3 the odd ones,
+      // 32 keys each: a warp has two tile times for every tile it computes
+      const int kb8 = (warp & 1) * 32;
+      if ((it & 1) == (warp >> 1) && kb8 < si.rows) {
         const float* sk = reinterpret_cast<const float*>(smem + s * C::kStageBytes + C::kScaleOff);
-        warp_tile_i8<D>(st, qf, smem_u32(smem + s * C::kStageBytes), sk, sk + kDecTileKeys, kb, si.rows, lane,
+        warp_tile_i8<D>(st, qf, smem_u32(smem + s * C::kStageBytes), sk, sk + kDecTileKeys, kb8, si.rows, lane,
                         p.scale_log2);
-      } else {
-        warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
       }
+    } else if (kb < si.rows) {
+      warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
