@@ -168,17 +168,22 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Four int8 codes (one 32-bit word, code i in byte i) -> two f16x2 holding
-// them exactly: lo = (code 0, code 1), hi = (code 2, code 3). Biased by 128 a
-// code is a byte u; the f16 with bits 0x64uu is 1024 + u (the 10-bit mantissa
-// holds u exactly), and subtracting 1152 (bits 0x6480) leaves the code.
-__device__ __forceinline__ void int8x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+// Int8 codes -> fp16 values code + 1152, exact: biased by 128 a code is a
+// byte u, and the fp16 with bits 0x64uu is 1024 + u (the 10-bit mantissa
+// holds u exactly). The caller takes the 1152 out of its sums.
+// Four codes of one word (code i in byte i): lo = (code 0, code 1), hi = (code 2, code 3).
+__device__ __forceinline__ void codes4_to_f16x2_biased(uint32_t w, uint32_t& lo, uint32_t& hi) {
   const uint32_t u = w ^ 0x80808080u;
-  const uint32_t blo = __byte_perm(u, 0x64646464u, 0x5140);  // bytes u0, 0x64, u1, 0x64
-  const uint32_t bhi = __byte_perm(u, 0x64646464u, 0x5342);  // bytes u2, 0x64, u3, 0x64
-  const uint32_t bias = 0x64806480u;
-  asm("sub.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(blo), "r"(bias));
-  asm("sub.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(bhi), "r"(bias));
+  lo = __byte_perm(u, 0x64646464u, 0x5140);  // bytes u0, 0x64, u1, 0x64
+  hi = __byte_perm(u, 0x64646464u, 0x5342);  // bytes u2, 0x64, u3, 0x64
+}
+
+// The same for a word (x0, y0, x1, y1) of two code pairs, as a transposing
+// ldmatrix of byte pairs delivers them: even = (x0, x1), odd = (y0, y1).
+__device__ __forceinline__ void code_pairs_to_f16x2_biased(uint32_t w, uint32_t& even, uint32_t& odd) {
+  const uint32_t u = w ^ 0x80808080u;
+  even = __byte_perm(u, 0x64646464u, 0x5240);  // bytes u0, 0x64, u2, 0x64
+  odd = __byte_perm(u, 0x64646464u, 0x5341);   // bytes u1, 0x64, u3, 0x64
 }
 
 // Transpose an 8x8 matrix of 16-bit values held as one m8n8 fragment per warp.

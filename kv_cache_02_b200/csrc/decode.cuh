@@ -315,10 +315,12 @@ __device__ __forceinline__ void load_q_frag(uint32_t (&qf)[D / 16][2], const __n
 template <int D>
 struct WarpState {
   float m_a, m_b, l_a, l_b;
+  float b_a, b_b;  // 8-bit path: sum of the fp16 P^T entries, the weight of the code bias in o
   float o[D / 16][4];
   __device__ __forceinline__ void reset() {
     m_a = m_b = -INFINITY;
     l_a = l_b = 0.f;
+    b_a = b_b = 0.f;
 #pragma unroll
     for (int md = 0; md < D / 16; ++md) o[md][0] = o[md][1] = o[md][2] = o[md][3] = 0.f;
   }
@@ -402,23 +404,48 @@ __device__ __forceinline__ void warp_tile(WarpState<D>& st, const uint32_t (&qf)
   }
 }
 
-// The 8-bit cache: one warp's 16 keys (kb .. kb+15) of the tile in `stage`
-// (codes), sk / sv the tile's K and V scales. Codes are exact in fp16: the
-// MMAs run fp16 x fp16 -> fp32, the K scale multiplies the score and the V
-// scale the probability (the softmax sums stay unscaled). A plain ldmatrix
-// gives a lane 4 consecutive codes of one key row: for Q K^T they are the
-// A operand with the head dims permuted as in load_q_frag_i8; for V^T P^T a
-// movmatrix transposes them into (dim, key pair) fragments, row m of a
-// 16-dim step d0 being dim d0 + i8_dim(m) (see stash_warp_state).
-__device__ __forceinline__ int i8_dim(int m) { return 4 * ((m & 7) >> 1) + (m & 1) + ((m >> 3) << 1); }
+// The 8-bit cache. Codes reach the MMAs as exact fp16 values biased by
+// kCodeBias (code + 1152: the fp16 with bits 0x64uu is 1024 + u for a byte u =
+// code + 128), fp16 x fp16 -> fp32; the bias is taken out of the sums
+// afterwards (one subtraction per score, one per output element) rather than
+// out of every code. The K scale multiplies the score and the V scale the
+// probability (the softmax sums stay unscaled).
+//   Q K^T: a plain ldmatrix gives a lane 4 consecutive codes of one key row,
+// the A operand with the head dims permuted as in load_q_frag_i8; the score
+// of key k for head h is S - kCodeBias * sum_d q_hd.
+//   V^T P^T: a transposing ldmatrix gives a lane the codes of dims 2g, 2g+1
+// for keys 2t, 2t+1 (g = lane/4, t = lane%4), so byte selects alone make the
+// A operand, row g of a 16-dim step d0 being dim d0 + 2g and row g + 8 dim
+// d0 + 2g + 1 (see stash_warp_state); o then holds O + kCodeBias * sum_k P_k.
+constexpr float kCodeBias = 1152.f;
+
+// kCodeBias * sum_d q_hd for this lane's score heads a = 2*(lane%4) and
+// b = a + 1, from the fp16 Q fragment of load_q_frag_i8 (the values the MMA
+// multiplies).
+template <int D>
+__device__ __forceinline__ void q_code_bias(const uint32_t (&qf)[D / 16][2], int lane, float& qb_a, float& qb_b) {
+  float sum = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&qf[ks][r]));
+      sum += f.x + f.y;
+    }
+  }
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);  // the four lanes of head lane/4
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  qb_a = kCodeBias * __shfl_sync(0xffffffffu, sum, 8 * (lane & 3));
+  qb_b = kCodeBias * __shfl_sync(0xffffffffu, sum, 8 * (lane & 3) + 4);
+}
 
 // One warp's 32 keys (kb .. kb+31) of the 8-bit tile in `stage`, as two
 // independent 16-key blocks (a: kb.., b: kb+16..) so that two MMA chains are
 // in flight; `rows` keys of the tile are valid, kb < rows.
 template <int D>
-__device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&qf)[D / 16][2], uint32_t stage_addr,
-                                             const float* sk, const float* sv, int kb, int rows, int lane,
-                                             float scale_log2) {
+__device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&qf)[D / 16][2], float qb_a,
+                                             float qb_b, uint32_t stage_addr, const float* sk, const float* sv,
+                                             int kb, int rows, int lane, float scale_log2) {
   using C = DecCfg<D, true>;
   const uint32_t k_base = stage_addr;
   const uint32_t v_base = stage_addr + C::kTileBytes;
@@ -426,7 +453,7 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
   const int row = kb + (lane & 7) + ((lane >> 3) & 1) * 8;
   const int ch = lane >> 4;
 
-  // S^T = K * Q^T for both blocks, two 16-dim steps per ldmatrix
+  // S^T + bias = K * Q^T for both blocks, two 16-dim steps per ldmatrix
   float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int j = 0; j < D / 32; ++j) {
@@ -436,8 +463,8 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
     uint32_t rl[4], rh[4], tl[4], th[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      int8x4_to_f16x2(r[i], rl[i], rh[i]);
-      int8x4_to_f16x2(t[i], tl[i], th[i]);
+      codes4_to_f16x2_biased(r[i], rl[i], rh[i]);
+      codes4_to_f16x2_biased(t[i], tl[i], th[i]);
     }
     mma_f16_16816(ca, rl[0], rl[1], rh[0], rh[1], qf[2 * j][0], qf[2 * j][1]);
     mma_f16_16816(cb, tl[0], tl[1], th[0], th[1], qf[2 * j][0], qf[2 * j][1]);
@@ -447,7 +474,7 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
 
   // online softmax over the 32 keys: key kb + lane/4 + 8 i for i = 0..3
   // (block a: c0/c1 and c2/c3, block b: the same, 16 keys on), each score
-  // scaled by its key's K scale
+  // unbiased and scaled by its key's K scale
   const int key0 = kb + (lane >> 2);
   bool vk[4];
   float xa[4], xb[4];
@@ -456,8 +483,8 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
     vk[i] = key0 + 8 * i < rows;
     const float sc = vk[i] ? sk[key0 + 8 * i] * scale_log2 : 0.f;
     const float* c = i < 2 ? ca : cb;
-    xa[i] = vk[i] ? c[2 * (i & 1)] * sc : -INFINITY;
-    xb[i] = vk[i] ? c[2 * (i & 1) + 1] * sc : -INFINITY;
+    xa[i] = vk[i] ? (c[2 * (i & 1)] - qb_a) * sc : -INFINITY;
+    xb[i] = vk[i] ? (c[2 * (i & 1) + 1] - qb_b) * sc : -INFINITY;
   }
   float mx_a = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
   float mx_b = fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3]));
@@ -486,34 +513,39 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
     st.o[md][3] *= al_b;
   }
 
-  // P^T times the V scales (keys past the valid rows: 0, their scales are never read)
+  // P^T times the V scales (keys past the valid rows: 0, their scales are
+  // never read), and the sums of those fp16 entries for the bias
   uint32_t pt[4];
+  float bs_a = 0.f, bs_b = 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float w = vk[i] ? sv[key0 + 8 * i] : 0.f;
-    pt[i] = movmatrix_trans(pack_f16x2(pa[i] * w, pb[i] * w));
+    const uint32_t pk = pack_f16x2(pa[i] * w, pb[i] * w);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pk));
+    bs_a += f.x;
+    bs_b += f.y;
+    pt[i] = movmatrix_trans(pk);
   }
+  st.b_a = st.b_a * al_a + bs_a;
+  st.b_b = st.b_b * al_b + bs_b;
 
-  // O^T += V^T * P^T for both blocks, two 16-dim steps per ldmatrix
+  // O^T + bias = V^T * P^T for both blocks, two 16-dim steps per ldmatrix:
+  // r[0]/r[1] keys 0-7 / 8-15 of the block for dims of step 2j, r[2]/r[3] of step 2j + 1
 #pragma unroll
   for (int j = 0; j < D / 32; ++j) {
     uint32_t r[4], t[4];
-    ldmatrix_x4(v_base + sw128(row, 2 * j + ch), r[0], r[1], r[2], r[3]);
-    ldmatrix_x4(v_base + sw128(row + 16, 2 * j + ch), t[0], t[1], t[2], t[3]);
-    uint32_t rl[4], rh[4], tl[4], th[4];
+    ldmatrix_x4_trans(v_base + sw128(row, 2 * j + ch), r[0], r[1], r[2], r[3]);
+    ldmatrix_x4_trans(v_base + sw128(row + 16, 2 * j + ch), t[0], t[1], t[2], t[3]);
+    uint32_t re[4], ro[4], te[4], to[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      int8x4_to_f16x2(r[i], rl[i], rh[i]);
-      int8x4_to_f16x2(t[i], tl[i], th[i]);
+      code_pairs_to_f16x2_biased(r[i], re[i], ro[i]);
+      code_pairs_to_f16x2_biased(t[i], te[i], to[i]);
     }
-    mma_f16_16816(st.o[2 * j], movmatrix_trans(rl[0]), movmatrix_trans(rh[0]), movmatrix_trans(rl[1]),
-                  movmatrix_trans(rh[1]), pt[0], pt[1]);
-    mma_f16_16816(st.o[2 * j + 1], movmatrix_trans(rl[2]), movmatrix_trans(rh[2]), movmatrix_trans(rl[3]),
-                  movmatrix_trans(rh[3]), pt[0], pt[1]);
-    mma_f16_16816(st.o[2 * j], movmatrix_trans(tl[0]), movmatrix_trans(th[0]), movmatrix_trans(tl[1]),
-                  movmatrix_trans(th[1]), pt[2], pt[3]);
-    mma_f16_16816(st.o[2 * j + 1], movmatrix_trans(tl[2]), movmatrix_trans(th[2]), movmatrix_trans(tl[3]),
-                  movmatrix_trans(th[3]), pt[2], pt[3]);
+    mma_f16_16816(st.o[2 * j], re[0], ro[0], re[1], ro[1], pt[0], pt[1]);
+    mma_f16_16816(st.o[2 * j + 1], re[2], ro[2], re[3], ro[3], pt[0], pt[1]);
+    mma_f16_16816(st.o[2 * j], te[0], to[0], te[1], to[1], pt[2], pt[3]);
+    mma_f16_16816(st.o[2 * j + 1], te[2], to[2], te[3], to[3], pt[2], pt[3]);
   }
 }
 
@@ -537,15 +569,32 @@ __device__ __forceinline__ void stash_warp_state(float* merge, const WarpState<D
     red_l[warp * 8 + ha + 1] = l_b;
   }
   // accumulator rows g and g + 8 of a 16-dim step: dims g and g + 8, or for
-  // the 8-bit path the dims its movmatrix fragments carry
+  // the 8-bit path dims 2g and 2g + 1, less the code bias times the P^T sums
   const int dr = lane >> 2;
-  const int da = kInt8 ? i8_dim(dr) : dr, db = kInt8 ? i8_dim(dr + 8) : dr + 8;
+  const int da = kInt8 ? 2 * dr : dr, db = kInt8 ? 2 * dr + 1 : dr + 8;
+  if constexpr (kInt8) {
+    float b_a = st.b_a, b_b = st.b_b;
 #pragma unroll
-  for (int md = 0; md < D / 16; ++md) {
-    ow[ha * D + md * 16 + da] = st.o[md][0];
-    ow[(ha + 1) * D + md * 16 + da] = st.o[md][1];
-    ow[ha * D + md * 16 + db] = st.o[md][2];
-    ow[(ha + 1) * D + md * 16 + db] = st.o[md][3];
+    for (int off = 4; off < 32; off <<= 1) {
+      b_a += __shfl_xor_sync(0xffffffffu, b_a, off);
+      b_b += __shfl_xor_sync(0xffffffffu, b_b, off);
+    }
+    const float c_a = kCodeBias * b_a, c_b = kCodeBias * b_b;
+#pragma unroll
+    for (int md = 0; md < D / 16; ++md) {
+      ow[ha * D + md * 16 + da] = st.o[md][0] - c_a;
+      ow[(ha + 1) * D + md * 16 + da] = st.o[md][1] - c_b;
+      ow[ha * D + md * 16 + db] = st.o[md][2] - c_a;
+      ow[(ha + 1) * D + md * 16 + db] = st.o[md][3] - c_b;
+    }
+  } else {
+#pragma unroll
+    for (int md = 0; md < D / 16; ++md) {
+      ow[ha * D + md * 16 + da] = st.o[md][0];
+      ow[(ha + 1) * D + md * 16 + da] = st.o[md][1];
+      ow[ha * D + md * 16 + db] = st.o[md][2];
+      ow[(ha + 1) * D + md * 16 + db] = st.o[md][3];
+    }
   }
 }
 
@@ -821,6 +870,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   const int tid = threadIdx.x;  // 0..127
   const int kb = warp * 16;
   uint32_t qf[D / 16][2];
+  float qb_a = 0.f, qb_b = 0.f;  // 8-bit path: the code bias of the scores
   WarpState<D> st;
   ItemCoord cur{};
   for (int it = 0;; ++it) {
@@ -831,9 +881,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (si.flags & kTileFirst) {
       cur = item_coord(p, si.item);
       const __nv_bfloat16* qh = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)cur.b * p.H + cur.h0) * D;
-      if constexpr (kInt8)
+      if constexpr (kInt8) {
         load_q_frag_i8<D>(qf, qh, lane, cur.nh);
-      else
+        q_code_bias<D>(qf, lane, qb_a, qb_b);
+      } else
         load_q_frag<D>(qf, qh, lane, cur.nh);
       st.reset();
     }
@@ -847,8 +898,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       const int kb8 = (warp & 1) * 32;
       if ((it & 1) == (warp >> 1) && kb8 < si.rows) {
         const float* sk = reinterpret_cast<const float*>(smem + s * C::kStageBytes + C::kScaleOff);
-        warp_tile_i8<D>(st, qf, smem_u32(smem + s * C::kStageBytes), sk, sk + kDecTileKeys, kb8, si.rows, lane,
-                        p.scale_log2);
+        warp_tile_i8<D>(st, qf, qb_a, qb_b, smem_u32(smem + s * C::kStageBytes), sk, sk + kDecTileKeys, kb8,
+                        si.rows, lane, p.scale_log2);
       }
     } else if (kb < si.rows) {
       warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
