@@ -52,8 +52,9 @@ struct DecCfg {
   static constexpr int kHalfBytes = kDecTileKeys * 128;        // one column box of a tile
   static constexpr int kTileBytes = kDecTileKeys * D * kElt;   // K (or V) tile
   static constexpr int kScaleOff = 2 * kTileBytes;             // 8-bit: K scales, then V scales
+  static constexpr int kQOff = kScaleOff + 2 * kDecTileKeys * 4;  // 8-bit: the item's q rows (first tile)
   static constexpr int kStages = kInt8 ? 5 : ((D == 128) ? 3 : 6);
-  static constexpr int kStageBytes = kInt8 ? (2 * kTileBytes + 2 * kDecTileKeys * 4 + 1023) / 1024 * 1024
+  static constexpr int kStageBytes = kInt8 ? (kQOff + kDecHeadsPerCta * D * 2 + 1023) / 1024 * 1024
                                            : 2 * kTileBytes;
   static constexpr int kRingBytes = kStages * kStageBytes;
   // merge scratch: per consumer warp, m and l of 8 heads, then O of 8 heads
@@ -244,16 +245,16 @@ __device__ __forceinline__ void issue_tile_i8(uint8_t* stage, uint64_t* full, co
                                               const CUtensorMap* tm_v64, const CUtensorMap* tm_k16,
                                               const CUtensorMap* tm_v16, const CUtensorMap* tm_ks,
                                               const CUtensorMap* tm_vs, int row0, int unit, int t0, int rows,
-                                              uint64_t policy) {
+                                              const void* q_rows, uint32_t q_bytes, uint64_t policy) {
   using C = DecCfg<D, true>;
   constexpr uint32_t kScaleBytes = kDecTileKeys * 4;
   if (rows == kDecTileKeys) {
-    mbar_arrive_expect_tx(full, (uint32_t)(2 * C::kTileBytes) + 2 * kScaleBytes);
+    mbar_arrive_expect_tx(full, (uint32_t)(2 * C::kTileBytes) + 2 * kScaleBytes + q_bytes);
     tma_load_2d(stage, tm_k64, 0, row0, full, policy);
     tma_load_2d(stage + C::kTileBytes, tm_v64, 0, row0, full, policy);
   } else {
     const int nbox = (rows + kDecBoxRows - 1) / kDecBoxRows;
-    mbar_arrive_expect_tx(full, (uint32_t)(nbox * kDecBoxRows * 128 * 2) + 2 * kScaleBytes);
+    mbar_arrive_expect_tx(full, (uint32_t)(nbox * kDecBoxRows * 128 * 2) + 2 * kScaleBytes + q_bytes);
     for (int bx = 0; bx < nbox; ++bx) {
       tma_load_2d(stage + bx * kDecBoxRows * 128, tm_k16, 0, row0 + bx * kDecBoxRows, full, policy);
       tma_load_2d(stage + C::kTileBytes + bx * kDecBoxRows * 128, tm_v16, 0, row0 + bx * kDecBoxRows, full, policy);
@@ -261,6 +262,7 @@ __device__ __forceinline__ void issue_tile_i8(uint8_t* stage, uint64_t* full, co
   }
   tma_load_2d(stage + C::kScaleOff, tm_ks, t0, unit, full, policy);
   tma_load_2d(stage + C::kScaleOff + kScaleBytes, tm_vs, t0, unit, full, policy);
+  if (q_bytes) bulk_load(stage + C::kQOff, q_rows, q_bytes, full);
 }
 
 // Table entries of the 16-row boxes of the tile of keys t0 .. t0 + rows - 1
@@ -275,12 +277,11 @@ __device__ __forceinline__ void tile_blocks(const DecodeParams& p, int b, int t0
     blk[bx] = bx * kDecBoxRows < rows ? __ldg(row + (t0 + bx * kDecBoxRows) / p.block_size) : 0;
 }
 
-// Q^T as the B operand (k = dims, n = heads): lane holds head lane/4, dims
-// 2*(lane%4) + {0,1} (b0) and + 8 (b1) of every 16-dim step.
-// Q^T as the fp16 B operand of the 8-bit path: in the 16-dim step ks the
-// lane holds head lane/4, dims 16 ks + 4 (lane%4) + {0, 1} (b0) and
-// + {2, 3} (b1) -- the order in which a key row's codes reach the A operand
-// (warp_tile_i8), so the dot products are unchanged.
+// Q^T as the fp16 B operand of the 8-bit path, from the item's q rows in
+// shared memory: in the 16-dim step ks the lane holds head lane/4, dims
+// 16 ks + 4 (lane%4) + {0, 1} (b0) and + {2, 3} (b1) -- the order in which a
+// key row's codes reach the A operand (warp_tile_i8), so the dot products
+// are unchanged.
 template <int D>
 __device__ __forceinline__ void load_q_frag_i8(uint32_t (&qf)[D / 16][2], const __nv_bfloat16* q, int lane, int nh) {
   const int hn = lane >> 2;
@@ -288,7 +289,7 @@ __device__ __forceinline__ void load_q_frag_i8(uint32_t (&qf)[D / 16][2], const 
   const uint2* qrow = reinterpret_cast<const uint2*>(q + (size_t)(hv ? hn : 0) * D);
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
-    const uint2 w = __ldg(qrow + ks * 4 + (lane & 3));
+    const uint2 w = qrow[ks * 4 + (lane & 3)];
     const float f0 = __uint_as_float(w.x << 16), f1 = __uint_as_float(w.x & 0xffff0000u);
     const float f2 = __uint_as_float(w.y << 16), f3 = __uint_as_float(w.y & 0xffff0000u);
     qf[ks][0] = hv ? pack_f16x2(f0, f1) : 0u;
@@ -296,6 +297,8 @@ __device__ __forceinline__ void load_q_frag_i8(uint32_t (&qf)[D / 16][2], const 
   }
 }
 
+// Q^T as the B operand (k = dims, n = heads): lane holds head lane/4, dims
+// 2*(lane%4) + {0,1} (b0) and + 8 (b1) of every 16-dim step.
 template <int D>
 __device__ __forceinline__ void load_q_frag(uint32_t (&qf)[D / 16][2], const __nv_bfloat16* q, int lane, int nh) {
   const int hn = lane >> 2;
@@ -439,13 +442,14 @@ __device__ __forceinline__ void q_code_bias(const uint32_t (&qf)[D / 16][2], int
   qb_b = kCodeBias * __shfl_sync(0xffffffffu, sum, 8 * (lane & 3) + 4);
 }
 
-// One warp's 32 keys (kb .. kb+31) of the 8-bit tile in `stage`, as two
-// independent 16-key blocks (a: kb.., b: kb+16..) so that two MMA chains are
-// in flight; `rows` keys of the tile are valid, kb < rows.
-template <int D>
+// One warp's NB x 16 keys (kb .. kb + 16 NB - 1) of the 8-bit tile in
+// `stage`: NB independent 16-key blocks, so that NB MMA chains are in
+// flight; `rows` keys of the tile are valid, kb < rows.
+template <int D, int NB>
 __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&qf)[D / 16][2], float qb_a,
                                              float qb_b, uint32_t stage_addr, const float* sk, const float* sv,
                                              int kb, int rows, int lane, float scale_log2) {
+  static_assert(NB == 1 || NB == 2, "one or two key blocks");
   using C = DecCfg<D, true>;
   const uint32_t k_base = stage_addr;
   const uint32_t v_base = stage_addr + C::kTileBytes;
@@ -453,41 +457,46 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
   const int row = kb + (lane & 7) + ((lane >> 3) & 1) * 8;
   const int ch = lane >> 4;
 
-  // S^T + bias = K * Q^T for both blocks, two 16-dim steps per ldmatrix
-  float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+  // S^T + bias = K * Q^T for each block, two 16-dim steps per ldmatrix
+  float c[NB][4];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) c[nb][0] = c[nb][1] = c[nb][2] = c[nb][3] = 0.f;
 #pragma unroll
   for (int j = 0; j < D / 32; ++j) {
-    uint32_t r[4], t[4];
-    ldmatrix_x4(k_base + sw128(row, 2 * j + ch), r[0], r[1], r[2], r[3]);
-    ldmatrix_x4(k_base + sw128(row + 16, 2 * j + ch), t[0], t[1], t[2], t[3]);
-    uint32_t rl[4], rh[4], tl[4], th[4];
+    uint32_t r[NB][4], lo[NB][4], hi[NB][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      codes4_to_f16x2_biased(r[i], rl[i], rh[i]);
-      codes4_to_f16x2_biased(t[i], tl[i], th[i]);
+    for (int nb = 0; nb < NB; ++nb) {
+      ldmatrix_x4(k_base + sw128(row + 16 * nb, 2 * j + ch), r[nb][0], r[nb][1], r[nb][2], r[nb][3]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) codes4_to_f16x2_biased(r[nb][i], lo[nb][i], hi[nb][i]);
     }
-    mma_f16_16816(ca, rl[0], rl[1], rh[0], rh[1], qf[2 * j][0], qf[2 * j][1]);
-    mma_f16_16816(cb, tl[0], tl[1], th[0], th[1], qf[2 * j][0], qf[2 * j][1]);
-    mma_f16_16816(ca, rl[2], rl[3], rh[2], rh[3], qf[2 * j + 1][0], qf[2 * j + 1][1]);
-    mma_f16_16816(cb, tl[2], tl[3], th[2], th[3], qf[2 * j + 1][0], qf[2 * j + 1][1]);
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+      mma_f16_16816(c[nb], lo[nb][0], lo[nb][1], hi[nb][0], hi[nb][1], qf[2 * j][0], qf[2 * j][1]);
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+      mma_f16_16816(c[nb], lo[nb][2], lo[nb][3], hi[nb][2], hi[nb][3], qf[2 * j + 1][0], qf[2 * j + 1][1]);
   }
 
-  // online softmax over the 32 keys: key kb + lane/4 + 8 i for i = 0..3
-  // (block a: c0/c1 and c2/c3, block b: the same, 16 keys on), each score
-  // unbiased and scaled by its key's K scale
+  // online softmax over the keys: key kb + lane/4 + 8 i for i < 2 NB (block
+  // i/2, accumulator entries c0/c1 for even i and c2/c3 for odd i), each
+  // score unbiased and scaled by its key's K scale
+  constexpr int NK = 2 * NB;
   const int key0 = kb + (lane >> 2);
-  bool vk[4];
-  float xa[4], xb[4];
+  bool vk[NK];
+  float xa[NK], xb[NK];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < NK; ++i) {
     vk[i] = key0 + 8 * i < rows;
     const float sc = vk[i] ? sk[key0 + 8 * i] * scale_log2 : 0.f;
-    const float* c = i < 2 ? ca : cb;
-    xa[i] = vk[i] ? (c[2 * (i & 1)] - qb_a) * sc : -INFINITY;
-    xb[i] = vk[i] ? (c[2 * (i & 1) + 1] - qb_b) * sc : -INFINITY;
+    xa[i] = vk[i] ? (c[i >> 1][2 * (i & 1)] - qb_a) * sc : -INFINITY;
+    xb[i] = vk[i] ? (c[i >> 1][2 * (i & 1) + 1] - qb_b) * sc : -INFINITY;
   }
-  float mx_a = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
-  float mx_b = fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3]));
+  float mx_a = fmaxf(xa[0], xa[1]), mx_b = fmaxf(xb[0], xb[1]);
+  if constexpr (NB == 2) {
+    mx_a = fmaxf(mx_a, fmaxf(xa[2], xa[3]));
+    mx_b = fmaxf(mx_b, fmaxf(xb[2], xb[3]));
+  }
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
@@ -497,14 +506,19 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
   const float al_a = fast_exp2(st.m_a - mn_a), al_b = fast_exp2(st.m_b - mn_b);
   st.m_a = mn_a;
   st.m_b = mn_b;
-  float pa[4], pb[4];
+  float pa[NK], pb[NK];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < NK; ++i) {
     pa[i] = fast_exp2(xa[i] - mn_a);
     pb[i] = fast_exp2(xb[i] - mn_b);
   }
-  st.l_a = st.l_a * al_a + ((pa[0] + pa[1]) + (pa[2] + pa[3]));
-  st.l_b = st.l_b * al_b + ((pb[0] + pb[1]) + (pb[2] + pb[3]));
+  float sa = pa[0] + pa[1], sb = pb[0] + pb[1];
+  if constexpr (NB == 2) {
+    sa += pa[2] + pa[3];
+    sb += pb[2] + pb[3];
+  }
+  st.l_a = st.l_a * al_a + sa;
+  st.l_b = st.l_b * al_b + sb;
 #pragma unroll
   for (int md = 0; md < D / 16; ++md) {
     st.o[md][0] *= al_a;
@@ -515,10 +529,10 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
 
   // P^T times the V scales (keys past the valid rows: 0, their scales are
   // never read), and the sums of those fp16 entries for the bias
-  uint32_t pt[4];
+  uint32_t pt[NK];
   float bs_a = 0.f, bs_b = 0.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < NK; ++i) {
     const float w = vk[i] ? sv[key0 + 8 * i] : 0.f;
     const uint32_t pk = pack_f16x2(pa[i] * w, pb[i] * w);
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pk));
@@ -529,23 +543,22 @@ __device__ __forceinline__ void warp_tile_i8(WarpState<D>& st, const uint32_t (&
   st.b_a = st.b_a * al_a + bs_a;
   st.b_b = st.b_b * al_b + bs_b;
 
-  // O^T + bias = V^T * P^T for both blocks, two 16-dim steps per ldmatrix:
-  // r[0]/r[1] keys 0-7 / 8-15 of the block for dims of step 2j, r[2]/r[3] of step 2j + 1
+  // O^T + bias = V^T * P^T for each block, two 16-dim steps per ldmatrix:
+  // r[0]/r[1] keys 0-7 / 8-15 of the block for the dims of step 2j, r[2]/r[3] of step 2j + 1
 #pragma unroll
   for (int j = 0; j < D / 32; ++j) {
-    uint32_t r[4], t[4];
-    ldmatrix_x4_trans(v_base + sw128(row, 2 * j + ch), r[0], r[1], r[2], r[3]);
-    ldmatrix_x4_trans(v_base + sw128(row + 16, 2 * j + ch), t[0], t[1], t[2], t[3]);
-    uint32_t re[4], ro[4], te[4], to[4];
+    uint32_t r[NB][4], ev[NB][4], od[NB][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      code_pairs_to_f16x2_biased(r[i], re[i], ro[i]);
-      code_pairs_to_f16x2_biased(t[i], te[i], to[i]);
+    for (int nb = 0; nb < NB; ++nb) {
+      ldmatrix_x4_trans(v_base + sw128(row + 16 * nb, 2 * j + ch), r[nb][0], r[nb][1], r[nb][2], r[nb][3]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) code_pairs_to_f16x2_biased(r[nb][i], ev[nb][i], od[nb][i]);
     }
-    mma_f16_16816(st.o[2 * j], re[0], ro[0], re[1], ro[1], pt[0], pt[1]);
-    mma_f16_16816(st.o[2 * j + 1], re[2], ro[2], re[3], ro[3], pt[0], pt[1]);
-    mma_f16_16816(st.o[2 * j], te[0], to[0], te[1], to[1], pt[2], pt[3]);
-    mma_f16_16816(st.o[2 * j + 1], te[2], to[2], te[3], to[3], pt[2], pt[3]);
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      mma_f16_16816(st.o[2 * j], ev[nb][0], od[nb][0], ev[nb][1], od[nb][1], pt[2 * nb], pt[2 * nb + 1]);
+      mma_f16_16816(st.o[2 * j + 1], ev[nb][2], od[nb][2], ev[nb][3], od[nb][3], pt[2 * nb], pt[2 * nb + 1]);
+    }
   }
 }
 
@@ -843,7 +856,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                                 rows, policy);
           else if constexpr (kInt8)
             issue_tile_i8<D>(smem + s * C::kStageBytes, &full[s], &tm_k64, &tm_v64, &tm_k, &tm_v, &tm_ks, &tm_vs,
-                             c.unit * p.S_max + t0, c.unit, t0, rows, policy);
+                             c.unit * p.S_max + t0, c.unit, t0, rows,
+                             static_cast<const __nv_bfloat16*>(p.q) + ((size_t)c.b * p.H + c.h0) * D,
+                             tt == 0 ? (uint32_t)(c.nh * D * 2) : 0u, policy);
           else
             issue_tile<D>(smem + s * C::kStageBytes, &full[s], &tm_k64, &tm_v64, &tm_k, &tm_v, c.unit * p.S_max + t0,
                           rows, policy);
@@ -871,6 +886,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   const int kb = warp * 16;
   uint32_t qf[D / 16][2];
   float qb_a = 0.f, qb_b = 0.f;  // 8-bit path: the code bias of the scores
+  int ti = 0;                    // 8-bit path: index of the tile in its work item
   WarpState<D> st;
   ItemCoord cur{};
   for (int it = 0;; ++it) {
@@ -881,9 +897,11 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (si.flags & kTileFirst) {
       cur = item_coord(p, si.item);
       const __nv_bfloat16* qh = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)cur.b * p.H + cur.h0) * D;
-      if constexpr (kInt8) {
-        load_q_frag_i8<D>(qf, qh, lane, cur.nh);
+      if constexpr (kInt8) {  // the producer brought the item's q rows with its first tile
+        load_q_frag_i8<D>(qf, reinterpret_cast<const __nv_bfloat16*>(smem + s * C::kStageBytes + C::kQOff), lane,
+                          cur.nh);
         q_code_bias<D>(qf, lane, qb_a, qb_b);
+        ti = 0;
       } else
         load_q_frag<D>(qf, qh, lane, cur.nh);
       st.reset();
@@ -893,14 +911,22 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         append_row<D, kPaged>(p, cur, smem + s * C::kStageBytes, si.new_row, lane);
     }
     if constexpr (kInt8) {
-      // warps 0-1 take the even tiles of the ring, warps 2-3 the odd ones,
-      // 32 keys each: a warp has two tile times for every tile it computes
-      const int kb8 = (warp & 1) * 32;
-      if ((it & 1) == (warp >> 1) && kb8 < si.rows) {
-        const float* sk = reinterpret_cast<const float*>(smem + s * C::kStageBytes + C::kScaleOff);
-        warp_tile_i8<D>(st, qf, qb_a, qb_b, smem_u32(smem + s * C::kStageBytes), sk, sk + kDecTileKeys, kb8,
-                        si.rows, lane, p.scale_log2);
+      // warps 0-1 take the even tiles of a work item and warps 2-3 the odd
+      // ones, 32 keys each, so that a warp has two tile times for every tile
+      // it computes; the last tile of an odd count goes to all four warps,
+      // 16 keys each. Which warp sums which keys follows from the item alone,
+      // not from the order in which CTAs take items.
+      const float* sk = reinterpret_cast<const float*>(smem + s * C::kStageBytes + C::kScaleOff);
+      const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
+      if ((si.flags & kTileLast) && (ti & 1) == 0) {
+        if (kb < si.rows)
+          warp_tile_i8<D, 1>(st, qf, qb_a, qb_b, sa, sk, sk + kDecTileKeys, kb, si.rows, lane, p.scale_log2);
+      } else if ((ti & 1) == (warp >> 1)) {
+        const int kb8 = (warp & 1) * 32;
+        if (kb8 < si.rows)
+          warp_tile_i8<D, 2>(st, qf, qb_a, qb_b, sa, sk, sk + kDecTileKeys, kb8, si.rows, lane, p.scale_log2);
       }
+      ++ti;
     } else if (kb < si.rows) {
       warp_tile<D>(st, qf, smem_u32(smem + s * C::kStageBytes), kb, si.rows, lane, p.scale_log2);
     }

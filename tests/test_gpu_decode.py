@@ -149,9 +149,27 @@ def test_decode_full_size_sampled(gqa, name):
     assert_close(got[sel[:, 0], sel[:, 1]], ref, name)
 
 
+@pytest.mark.parametrize("name", ["ragged_70b_decode_b32_h64_k8_d128_s1k_16k", "long_ctx_mqa_b1_h64_k1_d128_s131072"])
+def test_decode_repeats_bit_for_bit(gqa, name):
+    """The persistent CTAs take work items in a different order on every call;
+    the result must not depend on that order."""
+    w = synth.DECODE_WORKLOADS[name]
+    inp = synth.decode_inputs(w)
+    q, kc, vc, lens = dev(inp["q"]), dev(inp["k_cache"]), dev(inp["v_cache"]), dev(inp["seqlens"])
+    ws_bytes = gqa.gqa_decode_workspace_bytes(w.B, w.H, w.K, w.S_max, w.d, 0)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(4):
+        out = torch.full_like(q, float("nan"))
+        gqa.gqa_decode(out, q, kc, vc, lens, 1.0 / np.sqrt(w.d), 0, ws)
+        assert gqa.gqa_get_last_error() == (0, 0)
+        outs.append(host(out))
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+
+
 # ---------------------------------------------------------------------------
-# automatic splits: many splits per unit, and the in-kernel combine by the
-# last split to arrive
+# automatic splits: many splits per unit, and the combine of many partials
 
 AUTO = [
     # B, H, K, d, S_max, lens

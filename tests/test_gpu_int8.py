@@ -146,3 +146,23 @@ def test_int8_full_size_sampled(gqa, name):
     ref = oracle.decode_int8(inp["q"], inp["k_codes"], inp["k_scale"], inp["v_codes"], inp["v_scale"], inp["seqlens"],
                              scale, sel=sel)
     assert_close(got[sel[:, 0], sel[:, 1]], ref, name)
+
+
+def test_int8_decode_repeats_bit_for_bit(gqa):
+    """The persistent CTAs take work items in a different order on every call;
+    which warp sums which keys, and so the result, must not depend on it."""
+    inp = synth.int8_inputs("int8_ragged_70b_decode_b32_h64_k8_d128_s1k_16k")
+    B, H, d = inp["q"].shape
+    K, S_max = inp["k_codes"].shape[1:3]
+    t = {k: dev(inp[k]) for k in ("q", "k_codes", "k_scale", "v_codes", "v_scale", "seqlens")}
+    wsb = gqa.gqa_decode_int8_workspace_bytes(B, H, K, S_max, d, 0)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(4):
+        out = torch.full_like(t["q"], float("nan"))
+        gqa.gqa_decode_int8(out, t["q"], t["k_codes"], t["k_scale"], t["v_codes"], t["v_scale"], t["seqlens"],
+                            1.0 / np.sqrt(d), 0, ws)
+        assert gqa.gqa_get_last_error() == (0, 0)
+        outs.append(host(out))
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
