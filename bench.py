@@ -186,16 +186,13 @@ def bench_ours(args, rank, world, local):
     kv_bytes_layer = 2 * B * K * S * d * 2  # K and V, every row once
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        for layer in range(LAYERS):
-            if ev is not None:
-                ev[layer][0].record(stream)
+    layer_args = [(out[layer], q[layer], kc[layer], vc[layer], k_new[layer], v_new[layer]) for layer in range(LAYERS)]
+
+    def step():
+        for o, qq, k, v, kn, vn in layer_args:
             # the new token's K/V go into the cache at row pos, then every head
             # attends over pos + 1 keys: one fused pass per layer
-            gqa.gqa_decode_append(out[layer], q[layer], kc[layer], vc[layer], k_new[layer], v_new[layer], pos, scale,
-                                  0, ws)
-            if ev is not None:
-                ev[layer][1].record(stream)
+            gqa.gqa_decode_append(o, qq, k, v, kn, vn, pos, scale, 0, ws)
 
     for _ in range(args.warmup):
         step()
@@ -204,31 +201,44 @@ def bench_ours(args, rank, world, local):
     if status != (0, 0):
         raise RuntimeError(f"device error during warm-up: {status}")
 
+    # the step as a CUDA graph: the same 32 calls, captured once and replayed,
+    # so no launch waits on the host
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
     import torch.distributed as dist
 
-    dec_events = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(LAYERS)]
-                  for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
+    def timed(run, steps):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
         t0.record(stream)
-        for s in range(args.steps):
-            step(dec_events[s])
+        for _ in range(steps):
+            run()
         t1.record(stream)
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    local_ms = t0.elapsed_time(t1)
-    dec_ms = [dec_events[s][l][0].elapsed_time(dec_events[s][l][1]) for s in range(args.steps) for l in range(LAYERS)]
+        if world > 1:
+            dist.barrier()
+        return t0.elapsed_time(t1)
+
+    with ClockSampler(local) as clocks:
+        local_ms = timed(graph.replay, args.steps)
     status = gqa.gqa_get_last_error()
     if status != (0, 0):
         raise RuntimeError(f"device error in the timed region: {status}")
-
     max_ms, total_bytes = aggregate(local_ms, kv_bytes_layer * LAYERS * args.steps)
     value = total_bytes / (max_ms * 1e-3) / 1e9
     ms_per_step = max_ms / args.steps
+
+    # the same step with the 32 calls issued one by one from Python
+    eager_steps = max(3, min(args.steps, 50))
+    eager_ms, eager_bytes = aggregate(timed(step, eager_steps), kv_bytes_layer * LAYERS * eager_steps)
+    del graph
 
     # end to end through the public API: pinned host inputs in, result out, every step
     q_h = q.cpu().pin_memory()
@@ -260,7 +270,9 @@ def bench_ours(args, rank, world, local):
     d2h = out_h.numel() * out_h.element_size()
 
     peaks, peak_src = measured_peaks()
-    dec_avg_ms = statistics.fmean(dec_ms)
+    # every launch in the timed region is this call (decode kernel + combine):
+    # its average duration is the region over the calls, gaps included
+    dec_avg_ms = max_ms / (args.steps * LAYERS)
     achieved = kv_bytes_layer / (dec_avg_ms * 1e-3) / 1e9
     traffic = profiled_traffic("decode_bf16_llama3_8b_traffic",
                                ["kv_cache_02_b200/csrc/decode.cuh", "kv_cache_02_b200/csrc/common.cuh"])
@@ -270,13 +282,17 @@ def bench_ours(args, rank, world, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": B, "H": H, "K": K, "d": d, "context": S,
                    "layers_per_step": LAYERS, "kv_append_per_layer": "fused into the decode pass",
+                   "step": "the 32 gqa_decode_append calls captured once as a CUDA graph and replayed",
                    "l2": "inputs larger than L2: each step streams 32 distinct 256 MiB cache pairs (8 GiB)",
                    "parallelism": f"replicas x{world}", "num_splits": "auto"},
         "roofline": {"bound": "hbm", "kernel": "gqa_decode_append (decode_bf16_kernel with the append + decode_combine_kernel)",
                      "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "peak_source": peak_src,
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": traffic, "algorithmic_bytes_per_launch": kv_bytes_layer,
-                     "avg_launch_ms": round(dec_avg_ms, 5)},
+                     "avg_launch_ms": round(dec_avg_ms, 5),
+                     "avg_launch_from": "timed region / calls (every launch in it is this call)"},
+        "eager": {"value": round(eager_bytes / (eager_ms * 1e-3) / 1e9, 1), "unit": UNIT, "steps": eager_steps,
+                  "note": "the same step with the calls issued one by one from Python"},
         "e2e": {"value": round(e2e_bytes / (e2e_max_ms * 1e-3) / 1e9, 1), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "pinned-host q, k_new, v_new, pos copied in and out copied back every step; "
@@ -312,6 +328,41 @@ class L2Flush:
         self.r.max()
 
 
+def back_to_back_ms(make_call, nbytes: int, reps: int) -> float:
+    """Per-call ms of calls run back to back from a CUDA graph. make_call(i)
+    builds a call over input copy i; the graph cycles through enough copies
+    that together they hold at least twice the L2 size of distinct rows, so
+    no call finds the rows it reads in L2 (the inputs are larger than L2)."""
+    import torch
+
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    copies = min(16, max(1, -(-2 * l2 // max(nbytes, 1))))
+    calls = [make_call(i) for i in range(copies)]
+    n = copies * max(1, -(-16 // copies))  # at least 16 calls per replay
+    for c in calls:  # eager once: one-time setup outside the capture
+        c()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(n):
+            calls[i % copies]()
+    graph.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) / n)
+    del graph, calls
+    return statistics.median(times)
+
+
+BACK_TO_BACK = "calls back to back from a CUDA graph over rotating input copies (>= 2x L2 of distinct rows)"
+
+
 def extra_measurements(args, only=None):
     """Other workloads, rank 0 at N = 1: decode configs and the causal prefill."""
     import torch
@@ -330,27 +381,23 @@ def extra_measurements(args, only=None):
             t = torch.from_numpy(np.ascontiguousarray(a))
             return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).cuda()
 
-        q, kc, vc, lens = to_dev(inp["q"]), to_dev(inp["k_cache"]), to_dev(inp["v_cache"]), to_dev(inp["seqlens"])
+        q, lens = to_dev(inp["q"]), to_dev(inp["seqlens"])
         out = torch.empty_like(q)
         wsb = gqa.gqa_decode_workspace_bytes(w.B, w.H, w.K, w.S_max, w.d, 0)
         ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
-        flush = L2Flush()
         kv_bytes = int(inp["seqlens"].astype(np.int64).sum()) * w.K * w.d * 2 * 2
-        times = []
-        for it in range(args.warmup + (args.steps if only else 20)):
-            flush()  # evict the previous iteration's cache rows from L2
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            gqa.gqa_decode(out, q, kc, vc, lens, 1.0 / np.sqrt(w.d), 0, ws)
-            b.record()
-            torch.cuda.synchronize()
-            if it >= args.warmup:
-                times.append(a.elapsed_time(b))
-        ms = statistics.median(times)
+
+        def make_call(i):
+            kc, vc = to_dev(inp["k_cache"]), to_dev(inp["v_cache"])
+            return lambda: gqa.gqa_decode(out, q, kc, vc, lens, 1.0 / np.sqrt(w.d), 0, ws)
+
+        ms = back_to_back_ms(make_call, kv_bytes, args.steps if only else 20)
+        if gqa.gqa_get_last_error() != (0, 0):
+            raise RuntimeError(f"device error in {name}")
         gbs = kv_bytes / (ms * 1e-3) / 1e9
         res[name] = {"ms": round(ms, 5), "kv_bytes": kv_bytes, "GB/s": round(gbs, 1),
-                     "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "l2": "flushed (512 MiB write, then 512 MiB read)"}
-        del q, kc, vc, out, ws, flush
+                     "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "timing": BACK_TO_BACK}
+        del q, out, ws
         torch.cuda.empty_cache()
     # paged caches: the same workloads' values over randomly placed blocks
     for name in PAGED_EXTRA:
@@ -417,7 +464,7 @@ def paged_measurement(args, name, peaks, steps):
         t = torch.from_numpy(np.ascontiguousarray(a))
         return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).cuda()
 
-    q, kp, vp, table = to_dev(inp["q"]), to_dev(inp["k_pool"]), to_dev(inp["v_pool"]), to_dev(inp["block_table"])
+    q, table = to_dev(inp["q"]), to_dev(inp["block_table"])
     out = torch.empty_like(q)
     wsb = gqa.gqa_decode_paged_workspace_bytes(w.B, w.H, w.K, w.d, pw.block_size, table.shape[1], 0)
     ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
@@ -426,35 +473,25 @@ def paged_measurement(args, name, peaks, steps):
         pos, kn, vn = to_dev(inp["pos"]), to_dev(inp["k_new"]), to_dev(inp["v_new"])
         lens = inp["pos"].astype(np.int64) + 1
 
-        def call():
-            gqa.gqa_decode_append_paged(out, q, kp, vp, kn, vn, table, pos, scale, 0, ws)
+        def make_call(i):
+            kp, vp = to_dev(inp["k_pool"]), to_dev(inp["v_pool"])
+            return lambda: gqa.gqa_decode_append_paged(out, q, kp, vp, kn, vn, table, pos, scale, 0, ws)
     else:
         sl = to_dev(inp["seqlens"])
         lens = inp["seqlens"].astype(np.int64)
 
-        def call():
-            gqa.gqa_decode_paged(out, q, kp, vp, table, sl, scale, 0, ws)
+        def make_call(i):
+            kp, vp = to_dev(inp["k_pool"]), to_dev(inp["v_pool"])
+            return lambda: gqa.gqa_decode_paged(out, q, kp, vp, table, sl, scale, 0, ws)
     kv_bytes = int(lens.sum()) * w.K * w.d * 2 * 2
-    flush = L2Flush()
-    times = []
-    for it in range(args.warmup + steps):
-        flush()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        call()
-        b.record()
-        torch.cuda.synchronize()
-        if it >= args.warmup:
-            times.append(a.elapsed_time(b))
+    ms = back_to_back_ms(make_call, kv_bytes, steps)
     if gqa.gqa_get_last_error() != (0, 0):
         raise RuntimeError(f"device error in {name}")
-    ms = statistics.median(times)
     gbs = kv_bytes / (ms * 1e-3) / 1e9
     r = {"ms": round(ms, 5), "kv_bytes": kv_bytes, "GB/s": round(gbs, 1),
          "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "block_size": pw.block_size,
-         "call": "gqa_decode_append_paged" if w.append else "gqa_decode_paged",
-         "l2": "flushed (512 MiB write, then 512 MiB read)"}
-    del q, kp, vp, table, out, ws, flush
+         "call": "gqa_decode_append_paged" if w.append else "gqa_decode_paged", "timing": BACK_TO_BACK}
+    del q, table, out, ws
     torch.cuda.empty_cache()
     return r
 
@@ -473,31 +510,24 @@ def int8_measurement(args, name, peaks, steps):
         t = torch.from_numpy(np.ascontiguousarray(a))
         return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).cuda()
 
-    q, kc, ks, vc, vs = (to_dev(inp[k]) for k in ("q", "k_codes", "k_scale", "v_codes", "v_scale"))
-    sl = to_dev(inp["seqlens"])
+    q, sl = to_dev(inp["q"]), to_dev(inp["seqlens"])
     out = torch.empty_like(q)
     wsb = gqa.gqa_decode_int8_workspace_bytes(B, H, K, S_max, d, 0)
     ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
     kv_bytes = int(inp["seqlens"].astype(np.int64).sum()) * K * (d + 4) * 2
-    flush = L2Flush()
-    times = []
-    for it in range(args.warmup + steps):
-        flush()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        gqa.gqa_decode_int8(out, q, kc, ks, vc, vs, sl, 1.0 / np.sqrt(d), 0, ws)
-        b.record()
-        torch.cuda.synchronize()
-        if it >= args.warmup:
-            times.append(a.elapsed_time(b))
+
+    def make_call(i):
+        kc, ks, vc, vs = (to_dev(inp[k]) for k in ("k_codes", "k_scale", "v_codes", "v_scale"))
+        return lambda: gqa.gqa_decode_int8(out, q, kc, ks, vc, vs, sl, 1.0 / np.sqrt(d), 0, ws)
+
+    ms = back_to_back_ms(make_call, kv_bytes, steps)
     if gqa.gqa_get_last_error() != (0, 0):
         raise RuntimeError(f"device error in {name}")
-    ms = statistics.median(times)
     gbs = kv_bytes / (ms * 1e-3) / 1e9
     r = {"ms": round(ms, 5), "kv_bytes": kv_bytes, "GB/s": round(gbs, 1),
          "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "call": "gqa_decode_int8",
-         "bytes": "int8 codes + one float scale per row", "l2": "flushed (512 MiB write, then 512 MiB read)"}
-    del q, kc, ks, vc, vs, out, ws, flush
+         "bytes": "int8 codes + one float scale per row", "timing": BACK_TO_BACK}
+    del q, out, ws
     torch.cuda.empty_cache()
     return r
 

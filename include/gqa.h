@@ -121,6 +121,11 @@ GQA_API size_t gqa_decode_workspace_bytes(int B, int H, int K, int S_max, int d,
  *             bytes for the same shape and num_splits; may be NULL when that
  *             size is 0. Its contents need no initialisation. Two calls that
  *             share a workspace must not overlap on the GPU.
+ *
+ * The call may be captured into a CUDA graph (stream capture) and replayed:
+ * nothing is read back to the host, and the work counter the persistent
+ * kernel keeps in the workspace is left reset at the end of every launch.
+ * A replay reuses the pointers and sizes of the capture.
  */
 GQA_API int gqa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int B,
                int H, int K, int S_max, int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,

@@ -78,7 +78,7 @@ struct DecodeParams {
   void* k_cache_w;             // the caches, written at row pos[b]
   void* v_cache_w;
   int len_add;                 // 0 (decode) or 1 (decode after append)
-  unsigned long long* ws_queue;  // work-item counter of the persistent kernel: tag | count
+  unsigned long long* ws_queue;  // [2]: work-item counter of the persistent kernel and its exit counter (tag | count)
   int nitems;                  // B * K * nsplit * hslices
   const int32_t* seqlens;
   int B, H, K, S_max, G, hslices, chunk, nsplit;
@@ -124,6 +124,20 @@ __device__ __forceinline__ int take_ticket(unsigned long long* cnt, unsigned lon
   }
   raise_error(GQA_DEVERR_TIMEOUT);
   return 0;
+}
+
+// Called once per CTA after its last ticket (q[0] the counter, q[1] an exit
+// counter of the same kind): the last CTA out resets both words to tag 0,
+// which no call uses (call tags are odd), so that a launch that repeats its
+// tag -- a CUDA graph replay -- finds them unclaimed. The fences order every
+// CTA's tickets before its exit ticket, and all of them before the reset.
+__device__ __forceinline__ void leave_queue(unsigned long long* q, unsigned long long tag) {
+  __threadfence();
+  if (take_ticket(q + 1, tag) == (int)gridDim.x) {
+    __threadfence();
+    reinterpret_cast<volatile unsigned long long*>(q)[0] = 0ull;
+    reinterpret_cast<volatile unsigned long long*>(q)[1] = 0ull;
+  }
 }
 
 // Row of key t of KV head g in the [rows, D] view of a paged pool, key t
@@ -812,8 +826,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
       for (int k = 0;; ++k) {
         // the first item of each CTA is its block index; later ones come from the counter
-        const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + take_ticket(p.ws_queue, p.tag) - 1;
-        if (item < 0 || item >= p.nitems) break;
+        const int ticket = k == 0 ? 1 : take_ticket(p.ws_queue, p.tag);
+        const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + ticket - 1;
+        if (ticket <= 0 || item >= p.nitems) break;
         const ItemCoord c = item_coord(p, item);
         const int raw = __ldg(p.seqlens + c.b);
         const int len = valid_len(raw + p.len_add, p.S_max);
@@ -865,6 +880,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         }
         if (!ok) break;
       }
+      leave_queue(p.ws_queue, p.tag);
       // no more work: a record without loads ends the consumers' loop
       if (ok) {
         const int s = it % C::kStages;

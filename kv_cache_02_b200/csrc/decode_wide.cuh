@@ -302,8 +302,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       bool ok = true;
       for (int k = 0;; ++k) {
         // the first item of each CTA is its block index; later ones come from the counter
-        const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + take_ticket(p.ws_queue, p.tag) - 1;
-        if (item < 0 || item >= p.nitems) break;
+        const int ticket = k == 0 ? 1 : take_ticket(p.ws_queue, p.tag);
+        const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + ticket - 1;
+        if (ticket <= 0 || item >= p.nitems) break;
         const ItemCoord c = item_coord_n(p, item, kWideHeads);
         const int raw = k == 0 ? raw_first : __ldg(p.seqlens + c.b);
         const int len = valid_len(raw + p.len_add, p.S_max);
@@ -359,6 +360,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         }
         if (!ok) break;
       }
+      leave_queue(p.ws_queue, p.tag);
       if (ok) {
         const int s = it % C::kStages;
         if (it >= C::kStages) ok = mbar_wait_bounded(&kv_empty[s], ((it / C::kStages) - 1) & 1);

@@ -168,6 +168,33 @@ def test_decode_repeats_bit_for_bit(gqa, name):
         assert np.array_equal(o, outs[0])
 
 
+@pytest.mark.parametrize("name", ["llama3_8b_decode_b8_h32_k8_d128_s8192", "long_ctx_mqa_b1_h64_k1_d128_s131072"])
+def test_decode_graph_replay(gqa, name):
+    """gqa_decode captured in a CUDA graph and replayed with new queries gives
+    the eager call's bits: the persistent kernel's work counter in the
+    workspace is left reset by every launch, although a replay repeats it."""
+    w = synth.DECODE_WORKLOADS[name]
+    inp = synth.decode_inputs(w)
+    q, kc, vc, lens = dev(inp["q"]), dev(inp["k_cache"]), dev(inp["v_cache"]), dev(inp["seqlens"])
+    ws_bytes = gqa.gqa_decode_workspace_bytes(w.B, w.H, w.K, w.S_max, w.d, 0)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+    scale = 1.0 / np.sqrt(w.d)
+    out, ref = torch.empty_like(q), torch.empty_like(q)
+    gqa.gqa_decode(out, q, kc, vc, lens, scale, 0, ws)  # eager first: one-time attribute setup
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gqa.gqa_decode(out, q, kc, vc, lens, scale, 0, ws)
+    for rep in range(3):
+        q.copy_(dev(synth.normal((w.B, w.H, w.d), synth.BF16, w.seed, 20 + rep)))
+        out.fill_(float("nan"))
+        g.replay()
+        gqa.gqa_decode(ref, q, kc, vc, lens, scale, 0, ws)
+        assert gqa.gqa_get_last_error() == (0, 0)
+        assert np.array_equal(host(out), host(ref)), f"replay {rep}"
+    del g
+
+
 # ---------------------------------------------------------------------------
 # automatic splits: many splits per unit, and the combine of many partials
 

@@ -166,3 +166,32 @@ def test_int8_decode_repeats_bit_for_bit(gqa):
         outs.append(host(out))
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
+
+
+def test_int8_decode_graph_replay(gqa):
+    """gqa_decode_int8 captured in a CUDA graph and replayed gives the eager call's bits."""
+    inp = synth.int8_inputs("int8_llama3_8b_decode_b8_h32_k8_d128_s8192")
+    B, H, d = inp["q"].shape
+    K, S_max = inp["k_codes"].shape[1:3]
+    t = {k: dev(inp[k]) for k in ("q", "k_codes", "k_scale", "v_codes", "v_scale", "seqlens")}
+    wsb = gqa.gqa_decode_int8_workspace_bytes(B, H, K, S_max, d, 0)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
+    out, ref = torch.empty_like(t["q"]), torch.empty_like(t["q"])
+
+    def call(o):
+        gqa.gqa_decode_int8(o, t["q"], t["k_codes"], t["k_scale"], t["v_codes"], t["v_scale"], t["seqlens"],
+                            1.0 / np.sqrt(d), 0, ws)
+
+    call(out)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(out)
+    for rep in range(3):
+        t["q"].copy_(dev(synth.normal((B, H, d), synth.BF16, 0x1D, 20 + rep)))
+        out.fill_(float("nan"))
+        g.replay()
+        call(ref)
+        assert gqa.gqa_get_last_error() == (0, 0)
+        assert np.array_equal(host(out), host(ref)), f"replay {rep}"
+    del g
