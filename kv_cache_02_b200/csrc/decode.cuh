@@ -216,39 +216,6 @@ __device__ __forceinline__ void issue_tile(uint8_t* stage, uint64_t* full, const
   }
 }
 
-// The same for a paged cache: a full tile inside one block (block size a
-// multiple of 64) as 64-row boxes, otherwise each 16-row box at its own row;
-// blk holds the table entries of the boxes' keys (tile_blocks), loaded a
-// tile ahead.
-template <int D>
-__device__ __forceinline__ void issue_tile_paged(uint8_t* stage, uint64_t* full, const CUtensorMap* tm_k64,
-                                                 const CUtensorMap* tm_v64, const CUtensorMap* tm_k16,
-                                                 const CUtensorMap* tm_v16, const DecodeParams& p, int g, int t0,
-                                                 const int (&blk)[kDecTileKeys / kDecBoxRows], int rows,
-                                                 uint64_t policy) {
-  using C = DecCfg<D>;
-  if (rows == kDecTileKeys && p.block_size % kDecTileKeys == 0) {
-    issue_tile<D>(stage, full, tm_k64, tm_v64, tm_k16, tm_v16, paged_row(p, blk[0], g, t0), rows, policy);
-    return;
-  }
-  int brow[kDecTileKeys / kDecBoxRows];
-#pragma unroll
-  for (int bx = 0; bx < kDecTileKeys / kDecBoxRows; ++bx)
-    brow[bx] = bx * kDecBoxRows < rows ? paged_row(p, blk[bx], g, t0 + bx * kDecBoxRows) : 0;
-  const int nbox = (rows + kDecBoxRows - 1) / kDecBoxRows;
-  mbar_arrive_expect_tx(full, (uint32_t)(nbox * kDecBoxRows * 128 * C::kHalves * 2));
-#pragma unroll
-  for (int bx = 0; bx < kDecTileKeys / kDecBoxRows; ++bx) {
-    if (bx >= nbox) break;
-#pragma unroll
-    for (int hf = 0; hf < C::kHalves; ++hf) {
-      const int off = hf * C::kHalfBytes + bx * kDecBoxRows * 128;
-      tma_load_2d(stage + off, tm_k16, hf * 64, brow[bx], full, policy);
-      tma_load_2d(stage + C::kTileBytes + off, tm_v16, hf * 64, brow[bx], full, policy);
-    }
-  }
-}
-
 // The 8-bit cache: the codes of a full tile as one 64-row box each for K and
 // V, a partial tile as 16-row boxes; the tile's 64 K and 64 V scales as one
 // box each from the [units, S_max] scale arrays (a box reaching past a row's
@@ -277,18 +244,6 @@ __device__ __forceinline__ void issue_tile_i8(uint8_t* stage, uint64_t* full, co
   tma_load_2d(stage + C::kScaleOff, tm_ks, t0, unit, full, policy);
   tma_load_2d(stage + C::kScaleOff + kScaleBytes, tm_vs, t0, unit, full, policy);
   if (q_bytes) bulk_load(stage + C::kQOff, q_rows, q_bytes, full);
-}
-
-// Table entries of the 16-row boxes of the tile of keys t0 .. t0 + rows - 1
-// of sequence b (every block size is a multiple of 16, so a box never
-// straddles blocks): independent loads, consumed only when the tile is
-// issued, so that they are in flight while the producer waits for a stage.
-__device__ __forceinline__ void tile_blocks(const DecodeParams& p, int b, int t0, int rows,
-                                            int (&blk)[kDecTileKeys / kDecBoxRows]) {
-  const int32_t* row = p.block_table + (size_t)b * p.max_blocks;
-#pragma unroll
-  for (int bx = 0; bx < kDecTileKeys / kDecBoxRows; ++bx)
-    blk[bx] = bx * kDecBoxRows < rows ? __ldg(row + (t0 + bx * kDecBoxRows) / p.block_size) : 0;
 }
 
 // Q^T as the fp16 B operand of the 8-bit path, from the item's q rows in
@@ -775,6 +730,128 @@ __device__ __forceinline__ void append_row(const DecodeParams& p, const ItemCoor
   __syncwarp();
 }
 
+// Producer of the paged kernel: the whole warp. Lane 0 takes the tickets
+// and the stage waits; at an item's start the lanes load up to 32 of its
+// table entries at once (one coalesced load, lane j block j of the window),
+// and each tile's 16-row boxes are issued by as many lanes, each finding its
+// box's block with one shuffle. A tile inside one block (block size a
+// multiple of 64) is issued by lane 0 as one 64-row box per column half, as
+// for the contiguous cache.
+template <int D>
+__device__ __forceinline__ void produce_paged(const DecodeParams& p, uint8_t* smem, StageInfo* info, uint64_t* full,
+                                              uint64_t* empty, const CUtensorMap* tm_k64, const CUtensorMap* tm_v64,
+                                              const CUtensorMap* tm_k16, const CUtensorMap* tm_v16, int lane) {
+  using C = DecCfg<D>;
+  constexpr unsigned kAll = 0xffffffffu;
+  if (lane == 0) {
+    prefetch_tensormap(tm_k64);
+    prefetch_tensormap(tm_v64);
+    prefetch_tensormap(tm_k16);
+    prefetch_tensormap(tm_v16);
+  }
+  const uint64_t policy = l2_policy_evict_first();
+  const int bs = p.block_size;
+  const bool whole = bs % kDecTileKeys == 0;  // every full tile lies inside one block
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+  int it = 0;  // ring position
+  bool ok = true;
+  for (int k = 0;; ++k) {
+    // the first item of each CTA is its block index; later ones come from the counter
+    int ticket = 1;
+    if (k > 0) {
+      if (lane == 0) ticket = take_ticket(p.ws_queue, p.tag);
+      ticket = __shfl_sync(kAll, ticket, 0);
+    }
+    const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + ticket - 1;
+    if (ticket <= 0 || item >= p.nitems) break;
+    const ItemCoord c = item_coord(p, item);
+    const int raw = __ldg(p.seqlens + c.b);
+    const int len = valid_len(raw + p.len_add, p.S_max);
+    if (lane == 0 && c.g == 0 && c.split == 0 && c.hsl == 0) {
+      if (p.len_add ? (raw < 0 || raw >= p.S_max) : (len != raw))
+        raise_error(p.len_add ? GQA_DEVERR_APPEND_POS : GQA_DEVERR_SEQLEN);
+    }
+    const int t_begin = c.split * p.chunk;
+    const int t_end = min(len, t_begin + p.chunk);
+    if (t_begin >= t_end) {
+      if (c.split == 0) {  // an empty sequence: zeros for this item's heads
+        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)c.b * p.H + c.h0) * D);
+        for (int i = lane; i < c.nh * D / 8; i += 32) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      continue;
+    }
+    const int ntiles = (t_end - t_begin + kDecTileKeys - 1) / kDecTileKeys;
+    const int32_t* trow = p.block_table + (size_t)c.b * p.max_blocks;
+    const int blk_end = (t_end - 1) / bs + 1;  // the item's blocks: [t_begin / bs, blk_end)
+    int win = t_begin / bs;                    // lane j holds the entry of block win + j
+    int ent = win + lane < blk_end ? __ldg(trow + win + lane) : 0;
+    for (int tt = 0; tt < ntiles && ok; ++tt, ++it) {
+      const int s = it % C::kStages;
+      const int t0 = t_begin + tt * kDecTileKeys;
+      const int rows = min(kDecTileKeys, t_end - t0);
+      const int last_blk = (t0 + rows - 1) / bs;
+      if (last_blk >= win + 32) {  // the tile's blocks are past the window: the next 32
+        win = t0 / bs;
+        ent = win + lane < blk_end ? __ldg(trow + win + lane) : 0;
+      }
+      if (lane == 0 && it >= C::kStages) ok = mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1);
+      ok = __shfl_sync(kAll, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      uint8_t* stage = smem + s * C::kStageBytes;
+      if (whole && rows == kDecTileKeys) {
+        const int e = __shfl_sync(kAll, ent, t0 / bs - win);
+        if (lane == 0) {
+          const int new_row = (p.len_add && t0 <= len - 1 && len - 1 < t0 + rows) ? len - 1 - t0 : -1;
+          info[s] = StageInfo{item, rows,
+                              (tt == 0 ? kTileFirst : 0) | (tt == ntiles - 1 ? kTileLast : 0) |
+                                  (len <= p.chunk ? kUnitSingleSplit : 0),
+                              new_row};
+          issue_tile<D>(stage, &full[s], tm_k64, tm_v64, tm_k16, tm_v16, paged_row(p, e, c.g, t0), rows, policy);
+        }
+      } else {
+        // 16-row box bx (keys t0 + 16 bx ..) by lane bx; a box lies inside one block
+        const int nbox = (rows + kDecBoxRows - 1) / kDecBoxRows;
+        const int bx = lane < nbox ? lane : 0;
+        const int e = __shfl_sync(kAll, ent, (t0 + bx * kDecBoxRows) / bs - win);
+        if (lane == 0) {
+          const int new_row = (p.len_add && t0 <= len - 1 && len - 1 < t0 + rows) ? len - 1 - t0 : -1;
+          info[s] = StageInfo{item, rows,
+                              (tt == 0 ? kTileFirst : 0) | (tt == ntiles - 1 ? kTileLast : 0) |
+                                  (len <= p.chunk ? kUnitSingleSplit : 0),
+                              new_row};
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(nbox * kDecBoxRows * 128 * C::kHalves * 2));
+        }
+        __syncwarp();
+        if (lane < nbox) {
+          const int brow = paged_row(p, e, c.g, t0 + bx * kDecBoxRows);
+#pragma unroll
+          for (int hf = 0; hf < C::kHalves; ++hf) {
+            const int off = hf * C::kHalfBytes + bx * kDecBoxRows * 128;
+            tma_load_2d(stage + off, tm_k16, hf * 64, brow, &full[s], policy);
+            tma_load_2d(stage + C::kTileBytes + off, tm_v16, hf * 64, brow, &full[s], policy);
+          }
+        }
+      }
+    }
+    if (!ok) break;
+  }
+  if (lane == 0) {
+    leave_queue(p.ws_queue, p.tag);
+    // no more work: a record without loads ends the consumers' loop
+    if (ok) {
+      const int s = it % C::kStages;
+      if (it >= C::kStages) ok = mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1);
+      if (ok) {
+        info[s] = StageInfo{-1, 0, 0, 0};
+        mbar_arrive(&full[s]);
+        ++it;
+      }
+    }
+    // this CTA's own loads must land before the block may exit
+    for (int j = max(0, it - C::kStages); j < it; ++j) mbar_wait_bounded(&full[j % C::kStages], (j / C::kStages) & 1);
+  }
+}
+
 // kPaged: the cache is a paged pool; kInt8: the cache holds 8-bit codes and
 // per-row scales (tm_k*/tm_v* then map codes, tm_ks/tm_vs the scales; the
 // bf16 kernels ignore tm_ks/tm_vs).
@@ -811,7 +888,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
   if (warp == kDecConsumerWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if constexpr (kPaged) {
+      produce_paged<D>(p, smem, info, full, empty, &tm_k64, &tm_v64, &tm_k, &tm_v, lane);
+    } else if (lane == 0) {
       prefetch_tensormap(&tm_k64);
       prefetch_tensormap(&tm_v64);
       prefetch_tensormap(&tm_k);
@@ -847,18 +926,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           continue;
         }
         const int ntiles = (t_end - t_begin + kDecTileKeys - 1) / kDecTileKeys;
-        int blk[kDecTileKeys / kDecBoxRows], blk_next[kDecTileKeys / kDecBoxRows];
-        if constexpr (kPaged) tile_blocks(p, c.b, t_begin, min(kDecTileKeys, t_end - t_begin), blk_next);
         for (int tt = 0; tt < ntiles && ok; ++tt, ++it) {
           const int s = it % C::kStages;
           const int t0 = t_begin + tt * kDecTileKeys;
           const int rows = min(kDecTileKeys, t_end - t0);
-          if constexpr (kPaged) {  // this tile's table entries; the next tile's load during the wait
-#pragma unroll
-            for (int bx = 0; bx < kDecTileKeys / kDecBoxRows; ++bx) blk[bx] = blk_next[bx];
-            if (tt + 1 < ntiles)
-              tile_blocks(p, c.b, t0 + kDecTileKeys, min(kDecTileKeys, t_end - t0 - kDecTileKeys), blk_next);
-          }
           if (it >= C::kStages) ok = mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1);
           if (!ok) break;
           const int new_row = (p.len_add && t0 <= len - 1 && len - 1 < t0 + rows) ? len - 1 - t0 : -1;
@@ -866,10 +937,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                               (tt == 0 ? kTileFirst : 0) | (tt == ntiles - 1 ? kTileLast : 0) |
                                   (len <= p.chunk ? kUnitSingleSplit : 0),
                               new_row};
-          if constexpr (kPaged)
-            issue_tile_paged<D>(smem + s * C::kStageBytes, &full[s], &tm_k64, &tm_v64, &tm_k, &tm_v, p, c.g, t0, blk,
-                                rows, policy);
-          else if constexpr (kInt8)
+          if constexpr (kInt8)
             issue_tile_i8<D>(smem + s * C::kStageBytes, &full[s], &tm_k64, &tm_v64, &tm_k, &tm_v, &tm_ks, &tm_vs,
                              c.unit * p.S_max + t0, c.unit, t0, rows,
                              static_cast<const __nv_bfloat16*>(p.q) + ((size_t)c.b * p.H + c.h0) * D,
