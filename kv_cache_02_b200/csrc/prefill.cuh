@@ -27,6 +27,43 @@
 
 namespace gqa {
 
+// Three-input maximum, and two fp32 lanes per instruction (Blackwell's
+// paired FMA and add): the softmax's per-score arithmetic in half the
+// instructions.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (d0, d1) = (a0, a1) * (b, b) + (c, c), each lane rounded once
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %4};\n"
+      " mov.b64 rc, {%5, %5};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// (s0, s1) += (a0, a1)
+__device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
+  asm("{\n .reg .b64 rs, ra;\n mov.b64 rs, {%0, %1};\n mov.b64 ra, {%2, %3};\n"
+      " add.rn.f32x2 rs, rs, ra;\n mov.b64 {%0, %1}, rs;\n}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(a0), "f"(a1));
+}
+
+// Maximum of 64 values as a tree of three-input maxima (depth 4)
+__device__ __forceinline__ float max64(const float (&x)[64]) {
+  float t[22], u[8];
+#pragma unroll
+  for (int i = 0; i < 21; ++i) t[i] = fmax3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+  t[21] = x[63];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) u[i] = fmax3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+  u[7] = t[21];
+  return fmax3(fmax3(u[0], u[1], u[2]), fmax3(u[3], u[4], u[5]), fmaxf(u[6], u[7]));
+}
+
 constexpr int kPfBM = 128;  // query rows per CTA
 constexpr int kPfBN = 64;   // keys per tile
 constexpr int kPfStages = 2;
@@ -292,17 +329,11 @@ __global__ void __launch_bounds__(kPfThreads, 2)
       // tiles need no mask.
       const float sl2 = p.scale_log2;
       const bool pos_scale = sl2 > 0.f;  // the same in every thread
-      float mt = -INFINITY;
-      if (pos_scale && kmax >= kPfBN - 1) {
+      if (!(pos_scale && kmax >= kPfBN - 1)) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) mt = fmaxf(mt, x[c]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = c <= kmax ? (pos_scale ? x[c] : x[c] * sl2) : -INFINITY;
-          mt = fmaxf(mt, x[c]);
-        }
+        for (int c = 0; c < 64; ++c) x[c] = c <= kmax ? (pos_scale ? x[c] : x[c] * sl2) : -INFINITY;
       }
+      float mt = max64(x);
       const float xs = pos_scale ? sl2 : 1.f;  // scale still to apply to x
       mt *= xs;
       float alpha = 1.f;
@@ -313,15 +344,20 @@ __global__ void __launch_bounds__(kPfThreads, 2)
         rescale = j > 0;
         m_used = m_new;
       }
-      float sum = 0.f;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;  // four partial sums, two per paired add
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = fast_exp2(fmaf(x[2 * c], xs, -m_used));
-        const float p1 = fast_exp2(fmaf(x[2 * c + 1], xs, -m_used));
-        sum += p0 + p1;
+        float y0, y1;
+        fma2(y0, y1, x[2 * c], x[2 * c + 1], xs, -m_used);
+        const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+        if (c & 1)
+          add2(s2, s3, p0, p1);
+        else
+          add2(s0, s1, p0, p1);
         pk[c] = pack_bf16x2(p0, p1);
       }
+      const float sum = (s0 + s1) + (s2 + s3);
       l = l * alpha + sum;
       // P buffer and O are free once the previous tile's PV has finished
       if (j > 0) {
