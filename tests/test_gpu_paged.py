@@ -189,3 +189,35 @@ def test_paged_full_size_sampled(gqa, name):
     if w.append:  # the appended rows, bit for bit
         assert np.array_equal(host(kp)[table[np.arange(B), pos // pw.block_size], :, pos % pw.block_size],
                               inp["k_new"])
+
+
+def test_paged_decode_graph_replay(gqa):
+    """gqa_decode_append_paged captured in a CUDA graph and replayed gives the
+    eager call's bits (the warp-wide paged producer and the work counter's
+    reset at the end of every launch)."""
+    pw = synth.PAGED_WORKLOADS["paged_llama3_8b_decode_b8_h32_k8_d128_s8192_bs16"]
+    w = synth.DECODE_WORKLOADS[pw.base]
+    inp = synth.paged_inputs(pw)
+    B, H, K, d = w.B, w.H, w.K, w.d
+    kp, vp, table = dev(inp["k_pool"]), dev(inp["v_pool"]), dev(inp["block_table"])
+    q, kn, vn, pos = dev(inp["q"]), dev(inp["k_new"]), dev(inp["v_new"]), dev(inp["pos"])
+    ws = workspace(gqa.gqa_decode_paged_workspace_bytes(B, H, K, d, pw.block_size, table.shape[1], 0))
+    out, ref = torch.empty_like(q), torch.empty_like(q)
+    scale = 1.0 / np.sqrt(d)
+
+    def call(o):
+        gqa.gqa_decode_append_paged(o, q, kp, vp, kn, vn, table, pos, scale, 0, ws)
+
+    call(out)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(out)
+    for rep in range(3):
+        q.copy_(dev(synth.normal((B, H, d), synth.BF16, w.seed, 30 + rep)))
+        out.fill_(float("nan"))
+        g.replay()
+        call(ref)
+        assert gqa.gqa_get_last_error() == (0, 0)
+        assert np.array_equal(host(out), host(ref)), f"replay {rep}"
+    del g
