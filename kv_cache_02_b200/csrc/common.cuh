@@ -68,15 +68,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed. Returns false
-// (and raises GQA_DEVERR_TIMEOUT) if that takes longer than kWaitLimitNs.
+// (and raises GQA_DEVERR_TIMEOUT) if that takes longer than kWaitLimitNs
+// after the first 256 unsuccessful tries: the clock is read only every 256
+// tries, so a short wait never pays for a read of it.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  unsigned long long t0 = globaltimer_ns();
+  unsigned long long t0 = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
-      raise_error(GQA_DEVERR_TIMEOUT);
-      return false;
+    if ((it & 255u) == 0) {
+      const unsigned long long t = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = t;
+      } else if (t - t0 > kWaitLimitNs) {
+        raise_error(GQA_DEVERR_TIMEOUT);
+        return false;
+      }
     }
   }
 }
