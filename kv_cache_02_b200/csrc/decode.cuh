@@ -17,15 +17,21 @@
 //
 // The key axis of each (b, g) unit is cut into splits of `chunk` keys; a
 // work item is (b, g, split, head slice). bf16: persistent CTAs, two per SM;
-// each CTA's producer thread takes items from a tagged atomic counter in
-// unit order and streams their tiles through its ring without a break, so a
-// work item's epilogue (merging the four warps, writing the output or the
-// split's partial) overlaps the next item's loads, and late items go to
-// whichever CTA is free. The counter word carries a per-call tag next to the
-// count, so stale or uninitialised workspace contents read as "no items
-// taken yet": the workspace needs no initialisation. Units with more than
-// one split are merged by decode_combine_kernel (log-sum-exp), launched as a
-// programmatic dependent so that its launch overlaps the decode kernel.
+// each CTA's producer takes items from a tagged atomic counter, split-major
+// (split s of every unit before split s + 1), and streams their tiles
+// through its ring without a break, so a work item's epilogue (merging the
+// four warps, writing the output or the split's partial) overlaps the next
+// item's loads, and late items go to whichever CTA is free. The counter word
+// carries a per-call tag next to the count, so stale or uninitialised
+// workspace contents read as "no items taken yet": the workspace needs no
+// initialisation; the last CTA out resets it, so a CUDA graph replay, which
+// repeats the tag, finds it unclaimed. Units with more than one split are
+// merged by decode_combine_kernel (log-sum-exp), launched as a programmatic
+// dependent so that its launch overlaps the decode kernel.
+//
+// Paged caches: the producer is the whole warp (table entries loaded
+// together, one lane per 16-row box). 8-bit caches: the consumers turn codes
+// into fp16 and take 32 keys of alternate tiles each (warp_tile_i8).
 //
 // f32 path (float32 storage, small problems): plain FMA, one warp per head.
 #pragma once
