@@ -881,6 +881,20 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (threadIdx.x == 0) raise_error(GQA_DEVERR_TIMEOUT);
     return;
   }
+  // contiguous producer: the descriptors and the first item's length are
+  // requested before the set-up barrier, so their latency overlaps it
+  int raw_first = 0;
+  if (!kPaged && warp == kDecConsumerWarps && lane == 0) {
+    prefetch_tensormap(&tm_k64);
+    prefetch_tensormap(&tm_v64);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    if constexpr (kInt8) {
+      prefetch_tensormap(&tm_ks);
+      prefetch_tensormap(&tm_vs);
+    }
+    if ((int)blockIdx.x < p.nitems) raw_first = __ldg(p.seqlens + item_coord(p, blockIdx.x).b);
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -897,14 +911,6 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if constexpr (kPaged) {
       produce_paged<D>(p, smem, info, full, empty, &tm_k64, &tm_v64, &tm_k, &tm_v, lane);
     } else if (lane == 0) {
-      prefetch_tensormap(&tm_k64);
-      prefetch_tensormap(&tm_v64);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      if constexpr (kInt8) {
-        prefetch_tensormap(&tm_ks);
-        prefetch_tensormap(&tm_vs);
-      }
       const uint64_t policy = l2_policy_evict_first();
       int it = 0;  // ring position
       bool ok = true;
@@ -915,7 +921,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + ticket - 1;
         if (ticket <= 0 || item >= p.nitems) break;
         const ItemCoord c = item_coord(p, item);
-        const int raw = __ldg(p.seqlens + c.b);
+        const int raw = k == 0 ? raw_first : __ldg(p.seqlens + c.b);
         const int len = valid_len(raw + p.len_add, p.S_max);
         if (c.g == 0 && c.split == 0 && c.hsl == 0) {
           if (p.len_add ? (raw < 0 || raw >= p.S_max) : (len != raw)) {
