@@ -245,8 +245,8 @@ DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gq
   } else {
     // narrow groups: about eight small work items per SM (their partials are
     // small), twelve for bf16 batches of many units, where the finer items
-    // shorten the tail (split sweeps: the Llama-3-8B layer 1 % and the 70B
-    // ragged batch 2 % faster; the 8-bit consumers pay more per item and
+    // shorten the tail (split sweeps: the 70B ragged batch 2 % faster, the
+    // Llama-3-8B layer within 1 %; the 8-bit consumers pay more per item and
     // are slower with more); wide groups: about one item per SM, since a
     // 64-head partial is 32 KB; never below 256 keys per split
     const long long per_sm = (!int8 && units >= 32) ? 12 : 8;
