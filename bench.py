@@ -202,9 +202,10 @@ def bench_ours(args, rank, world, local):
         raise RuntimeError(f"device error during warm-up: {status}")
 
     # the step as a CUDA graph: the same 32 calls, captured once and replayed,
-    # so no launch waits on the host
+    # so no launch waits on the host. Thread-local capture: other threads of
+    # the process (a process group's watchdog) may keep using CUDA meanwhile.
     graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
         step()
     for _ in range(args.warmup):
         graph.replay()
@@ -374,7 +375,7 @@ def back_to_back_ms(make_call, nbytes: int, reps: int) -> float:
         c()
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
         for i in range(n):
             calls[i % copies]()
     graph.replay()
