@@ -205,3 +205,25 @@ def test_oracle_and_cuda_path_share_no_code():
             assert "kv_cache_02_b200" not in _python_imports(p), p
         if f.endswith(".c"):
             assert "#include \"" not in open(p, encoding="utf-8").read(), p
+
+
+def test_binding_refuses_host_tensors(lib):
+    """There is no CPU path: the binding raises on host tensors instead of computing anything."""
+    import torch
+
+    from kv_cache_02_b200 import gqa
+
+    B, H, K, S, d = 2, 8, 2, 64, 64
+    q = torch.zeros((B, H, d), dtype=torch.bfloat16)
+    kc = torch.zeros((B, K, S, d), dtype=torch.bfloat16)
+    lens = torch.full((B,), S, dtype=torch.int32)
+    calls = [
+        lambda: gqa.gqa_decode(torch.empty_like(q), q, kc, kc, lens, 0.125),
+        lambda: gqa.gqa_decode_append(torch.empty_like(q), q, kc, kc, kc[:, :, 0], kc[:, :, 0], lens, 0.125),
+        lambda: gqa.gqa_kv_append(kc, kc, kc[:, :, 0], kc[:, :, 0], lens),
+        lambda: gqa.gqa_meanpool_kv(torch.empty((1, K, 16), dtype=torch.bfloat16),
+                                    torch.zeros((1, H, 16), dtype=torch.bfloat16)),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="on the GPU"):
+            call()
