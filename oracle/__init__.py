@@ -49,8 +49,9 @@ Page citations (title, section):
     i * block_size .. (i + 1) * block_size - 1. A paged decode is, by that
     definition, the decode of the cache the table gathers.
 
-Parity status: pinned (tests/test_oracle_pins.py); nothing here is "parity
-unpinned".
+Parity status: every function is pinned by a CPU test (tests/test_oracle_pins.py,
+tests/test_oracle_cache_write_pins.py and the paged, 8-bit, projection and
+varlen pin files); nothing here is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -335,11 +336,6 @@ def quantize_int8(x, lib=None):
     if rows:
         _get(lib).ref_quantize_int8(codes.ctypes.data, scales.ctypes.data, x.ctypes.data, _dtype_code(x), rows, n)
     return codes, scales
-
-
-def dequantize_int8(codes, scales) -> np.ndarray:
-    """code * scale in float64 (exact)."""
-    return codes.astype(np.float64) * scales.astype(np.float64)[..., None]
 
 
 def decode_int8(q, k_codes, k_scales, v_codes, v_scales, seqlens, scale: float, sel=None, nthreads=None,
