@@ -395,6 +395,132 @@ def back_to_back_ms(make_call, nbytes: int, reps: int) -> float:
 BACK_TO_BACK = "calls back to back from a CUDA graph over rotating input copies (>= 2x L2 of distinct rows)"
 
 
+def isolated_ms(make_call, reps: int, n: int = 16) -> float:
+    """Per-call ms of calls that each follow an L2 flush, so that no call
+    overlaps another or finds its rows in L2: a CUDA graph of n (flush, call)
+    pairs less a graph of n flushes alone, over n."""
+    import torch
+
+    flush = L2Flush()
+    call = make_call(0)
+    call()
+    torch.cuda.synchronize()
+    graphs = []
+    for with_call in (True, False):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for _ in range(n):
+                flush()
+                if with_call:
+                    call()
+        graphs.append(g)
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    diffs = []
+    for _ in range(reps):
+        t = []
+        for g in graphs:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            t.append(a.elapsed_time(b))
+        diffs.append((t[0] - t[1]) / n)
+    del graphs, flush
+    return statistics.median(diffs)
+
+
+ISOLATED = "each call after an L2 flush (a graph of flush + call pairs less a graph of flushes, per call)"
+
+KV_APPEND = "kv_append_b8_k8_d128_s8192"
+PROMPT_WRITE = "prompt_cache_write_b4_s4096_k8_d128"
+MEANPOOL = "meanpool_kv_h64_k8_d128_dm8192"
+SMALL_EXTRA = [KV_APPEND, PROMPT_WRITE, MEANPOOL]
+
+
+def small_kernel_measurements(args, peaks, steps, only=None):
+    """The HBM-bound kernels beside the decode: the append of one token (latency), the prompt's
+    K/V written to the cache (the bulk form of the append), and mean pooling of K/V projection
+    weights from 64 heads to 8."""
+    import torch
+
+    from kv_cache_02_b200 import gqa
+
+    res = {}
+    if only in (None, KV_APPEND):
+        # gqa_kv_append at the Llama-3-8B decode layer's shape: 2 B K rows of 256 bytes
+        B, K, d, S_max = 8, 8, 128, 8192
+        kn = torch.randn((B, K, d), device="cuda").to(torch.bfloat16)
+        vn = torch.randn((B, K, d), device="cuda").to(torch.bfloat16)
+        pos = torch.full((B,), S_max - 1, dtype=torch.int32, device="cuda")
+
+        def make_call(i):
+            kc = torch.empty((B, K, S_max, d), dtype=torch.bfloat16, device="cuda")
+            vc = torch.empty_like(kc)
+            return lambda: gqa.gqa_kv_append(kc, vc, kn, vn, pos)
+
+        ms = back_to_back_ms(make_call, 256 << 20, steps)
+        byts = 2 * 2 * B * K * d * 2  # the new rows read, and written into the caches
+        res[KV_APPEND] = {"ms": round(ms, 5), "bytes": byts, "GB/s": round(byts / (ms * 1e-3) / 1e9, 1),
+                          "bound": "launch latency (64 KiB moved)", "timing": "calls back to back from a CUDA graph"}
+        del kn, vn, pos
+    if only in (None, PROMPT_WRITE):
+        # the prompt's K/V [B,S,K,d] into the caches [B,K,S_max,d]: the causal prefill with the cache
+        # write less the prefill without it, each after an L2 flush
+        w = synth.PREFILL_WORKLOADS[PREFILL]
+        q = torch.randn((w.B, w.S, w.H, w.d), device="cuda").to(torch.bfloat16)
+        k = torch.randn((w.B, w.S, w.K, w.d), device="cuda").to(torch.bfloat16)
+        v = torch.randn_like(k)
+        out = torch.empty_like(q)
+        kc = torch.empty((w.B, w.K, w.S, w.d), dtype=torch.bfloat16, device="cuda")
+        vc = torch.empty_like(kc)
+        flush = L2Flush()
+        t = {True: [], False: []}
+        for it in range(args.warmup + steps):
+            for with_cache in (True, False):
+                flush()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                if with_cache:
+                    gqa.gqa_prefill_causal(out, q, k, v, 1.0 / np.sqrt(w.d), kc, vc)
+                else:
+                    gqa.gqa_prefill_causal(out, q, k, v, 1.0 / np.sqrt(w.d))
+                b.record()
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    t[with_cache].append(a.elapsed_time(b))
+        ms = statistics.median(t[True]) - statistics.median(t[False])
+        byts = 2 * 2 * w.B * w.S * w.K * w.d * 2  # K and V read once and written once
+        gbs = byts / (ms * 1e-3) / 1e9 if ms > 0 else None
+        res[PROMPT_WRITE] = {"ms": round(ms, 5), "bytes": byts, "GB/s": None if gbs is None else round(gbs, 1),
+                             "frac_of_measured_hbm": None if gbs is None else round(gbs / peaks["hbm_gbs"], 4),
+                             "timing": "gqa_prefill_causal with the cache write less without it, medians, "
+                                       "each call after an L2 flush"}
+        del q, k, v, out, kc, vc, flush
+    if only in (None, MEANPOOL):
+        # W_K of 64 heads [64, 128, 8192] -> 8 KV heads: 128 MiB read, 16 MiB written
+        H, K, d, dm = 64, 8, 128, 8192
+        dst = torch.empty((1, K, d * dm), dtype=torch.bfloat16, device="cuda")
+
+        def make_call(i):
+            src = torch.randn((1, H, d * dm), device="cuda").to(torch.bfloat16)
+            return lambda: gqa.gqa_meanpool_kv(dst, src)
+
+        src_bytes = H * d * dm * 2
+        ms = back_to_back_ms(make_call, src_bytes, steps)
+        byts = src_bytes + K * d * dm * 2
+        gbs = byts / (ms * 1e-3) / 1e9
+        res[MEANPOOL] = {"ms": round(ms, 5), "bytes": byts, "GB/s": round(gbs, 1),
+                         "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "timing": BACK_TO_BACK}
+        del dst
+    if gqa.gqa_get_last_error() != (0, 0):
+        raise RuntimeError("device error in the small-kernel measurements")
+    torch.cuda.empty_cache()
+    return res
+
+
 def extra_measurements(args, only=None):
     """Other workloads, rank 0 at N = 1: decode configs and the causal prefill."""
     import torch
@@ -429,6 +555,11 @@ def extra_measurements(args, only=None):
         gbs = kv_bytes / (ms * 1e-3) / 1e9
         res[name] = {"ms": round(ms, 5), "kv_bytes": kv_bytes, "GB/s": round(gbs, 1),
                      "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "timing": BACK_TO_BACK}
+        if kv_bytes < 256 << 20:  # a short call: also timed on its own
+            ims = isolated_ms(make_call, args.steps if only else 10)
+            igbs = kv_bytes / (ims * 1e-3) / 1e9
+            res[name]["isolated"] = {"ms": round(ims, 5), "GB/s": round(igbs, 1),
+                                     "frac_of_measured_hbm": round(igbs / peaks["hbm_gbs"], 4), "timing": ISOLATED}
         del q, out, ws
         torch.cuda.empty_cache()
     # paged caches: the same workloads' values over randomly placed blocks
@@ -448,6 +579,8 @@ def extra_measurements(args, only=None):
         if only is not None and name != only:
             continue
         res[name] = proj_measurement(args, name, peaks, 20 if only is None else args.steps)
+    if only is None or only in SMALL_EXTRA:
+        res.update(small_kernel_measurements(args, peaks, 20 if only is None else args.steps, only))
     if only is not None and only != PREFILL:
         return res
     # causal prefill with the KV-cache write: FLOPs over the causal pairs (j <= i) only
@@ -705,7 +838,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads and the CPU baseline")
-    ap.add_argument("--only", choices=DECODE_EXTRA + PAGED_EXTRA + INT8_EXTRA + VARLEN_EXTRA + PROJ_EXTRA + [PREFILL],
+    ap.add_argument("--only", choices=DECODE_EXTRA + PAGED_EXTRA + INT8_EXTRA + VARLEN_EXTRA + PROJ_EXTRA + SMALL_EXTRA
+                    + [PREFILL],
                     default=None,
                     help="time one other workload alone (for profiling); prints its own JSON, not the contract line")
     ap.add_argument("--layers", type=int, default=32,

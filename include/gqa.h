@@ -173,8 +173,15 @@ GQA_API int gqa_decode_append(void* out, const void* q, void* k_cache, void* v_c
  *    is rejected with GQA_ERR_SCRATCH_LIMIT before anything is launched; a
  *    smaller num_splits needs less scratch.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current). Make that first call
- *    before any stream capture begins on the device.
+ *    (cudaGetSymbolAddress, with that device current). Under CUDA's lazy
+ *    module loading (the default since CUDA 12.2) that lookup may load the
+ *    part of the library that holds the array: it reserves the
+ *    GQA_NOALLOC_SCRATCH_BYTES and can synchronise the device, as an
+ *    allocation would. Make one call per device at start-up, before any
+ *    stream capture begins on the device.
+ *  - A device reset (cudaDeviceReset) ends the context the address belongs
+ *    to. The next call sees that the device's context changed and looks the
+ *    address up again (which again loads the module, as above).
  *  - Every call on a device uses the same array, which keeps whatever the
  *    last call left in it. Calls that overlap on the GPU (unordered streams)
  *    race on it and produce wrong results: order them on one stream or with

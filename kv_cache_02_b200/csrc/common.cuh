@@ -22,8 +22,12 @@ __device__ unsigned int g_error_word;
 
 __device__ __forceinline__ void raise_error(unsigned int bit) { atomicOr(&g_error_word, bit); }
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer.
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+// A bounded wait gives up after this many nanoseconds of %globaltimer (1 s;
+// the wait-test build of the library sets a shorter limit).
+#ifndef GQA_WAIT_LIMIT_NS
+#define GQA_WAIT_LIMIT_NS 1000000000ull
+#endif
+constexpr unsigned long long kWaitLimitNs = GQA_WAIT_LIMIT_NS;
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
@@ -217,6 +221,61 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ---------------------------------------------------------------------------
+// programmatic dependent launch and L2 warm-up
+
+// Wait until the kernels this grid depends on (the previous kernel on the
+// stream, when this one was launched with programmatic stream serialization)
+// have finished and their memory operations are visible. A no-op otherwise.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next kernel on the stream, if launched as a programmatic
+// dependent, to be scheduled once every CTA of this grid has got here (or
+// exited).
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Ask L2 to fetch `bytes` contiguous bytes from global memory (address
+// 16-byte aligned, bytes a multiple of 16). A hint only: nothing is
+// delivered to the CTA, and a later load of the same bytes reads whatever L2
+// then holds, so it may run before the producer of those bytes has finished.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// host: kernel launch
+
+// Launch `kernel` on `st` with `smem` bytes of dynamic shared memory.
+// cudaLaunchKernelEx returns this launch's own error, so an error that the
+// caller left pending is neither reported as this launch's nor cleared; this
+// launch's error is cleared only if none was pending before it.
+// pdl: programmatic stream serialization. The kernel may then be scheduled
+// while the previous kernel on the stream is still running; every kernel
+// launched so here executes grid_dep_wait() in all of its threads before it
+// reads an input, writes an output or exits.
+template <typename... KArgs, typename... Args>
+inline int launch_kernel(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                         bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  const cudaError_t before = cudaPeekAtLastError();
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess) return GQA_OK;
+  if (before == cudaSuccess) cudaGetLastError();
+  return GQA_ERR_CUDA;
 }
 
 }  // namespace gqa

@@ -858,6 +858,37 @@ __device__ __forceinline__ void produce_paged(const DecodeParams& p, uint8_t* sm
   }
 }
 
+// Keys of a CTA's first work item that it asks L2 for before its grid
+// dependency resolves (K and V: 2 x 64 x 256 B = 32 KB per CTA for bf16
+// d = 128), so that the DRAM reads of a decode call start while the kernel
+// before it (the previous call's split combine, the tail of its decode)
+// finishes.
+#ifndef GQA_DEC_WARM_KEYS
+#define GQA_DEC_WARM_KEYS 192
+#endif
+constexpr int kDecWarmKeys = GQA_DEC_WARM_KEYS;
+
+// L2 warm-up of the first `max_keys` keys of work item `c` of a contiguous
+// cache ([units * S_max] rows of kRowBytes): K and V rows from the item's
+// first key, as far as the (possibly stale) length `raw` reaches. One head
+// slice per unit asks; the others read the same rows.
+template <int kRowBytes>
+__device__ __forceinline__ void warm_first_item(const DecodeParams& p, const ItemCoord& c, int raw, int max_keys) {
+  if (c.hsl != 0) return;
+  const int len = valid_len(raw + p.len_add, p.S_max);
+  const int t_begin = c.split * p.chunk;
+  const int t_end = min(min(len, t_begin + p.chunk), t_begin + max_keys);
+  if (t_end <= t_begin) return;
+  const size_t off = ((size_t)c.unit * p.S_max + t_begin) * kRowBytes;
+  const uint32_t bytes = (uint32_t)(t_end - t_begin) * kRowBytes;
+  constexpr uint32_t kStep = 32768;  // bytes per prefetch instruction
+  for (uint32_t o = 0; o < bytes; o += kStep) {
+    const uint32_t n = min(kStep, bytes - o);
+    prefetch_l2_bulk(static_cast<const uint8_t*>(p.k_cache_w) + off + o, n);
+    prefetch_l2_bulk(static_cast<const uint8_t*>(p.v_cache_w) + off + o, n);
+  }
+}
+
 // kPaged: the cache is a paged pool; kInt8: the cache holds 8-bit codes and
 // per-row scales (tm_k*/tm_v* then map codes, tm_ks/tm_vs the scales; the
 // bf16 kernels ignore tm_ks/tm_vs).
@@ -878,12 +909,17 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   const int lane = threadIdx.x & 31;
 
   if (smem_u32(smem) & 1023u) {  // the swizzle pattern needs 1024-byte aligned stages
+    grid_dep_wait();
     if (threadIdx.x == 0) raise_error(GQA_DEVERR_TIMEOUT);
     return;
   }
-  // contiguous producer: the descriptors and the first item's length are
-  // requested before the set-up barrier, so their latency overlaps it
-  int raw_first = 0;
+  // Launched as a programmatic dependent: until grid_dep_wait() returns, the
+  // previous kernel on the stream may still be running. Before it: the
+  // barriers, the descriptor prefetch, and (contiguous caches) an L2 warm-up
+  // of the first work item's key rows, sized by a length read that may be
+  // stale -- a hint only, so the rows may still be being written. After it
+  // the length is read again and every input is read for real.
+  int spec_first = 0;
   if (!kPaged && warp == kDecConsumerWarps && lane == 0) {
     prefetch_tensormap(&tm_k64);
     prefetch_tensormap(&tm_v64);
@@ -893,7 +929,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       prefetch_tensormap(&tm_ks);
       prefetch_tensormap(&tm_vs);
     }
-    if ((int)blockIdx.x < p.nitems) raw_first = __ldg(p.seqlens + item_coord(p, blockIdx.x).b);
+    // through L2 only (ld.cg): no L1 line of the possibly stale value survives the wait
+    if ((int)blockIdx.x < p.nitems) spec_first = __ldcg(p.seqlens + item_coord(p, blockIdx.x).b);
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -903,8 +940,11 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     fence_mbar_init();
   }
   __syncthreads();
-  // the combine kernel may be scheduled now; it waits for this grid to finish
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (!kPaged && warp == kDecConsumerWarps && lane == 0 && (int)blockIdx.x < p.nitems)
+    warm_first_item<D * C::kElt>(p, item_coord(p, blockIdx.x), spec_first, kDecWarmKeys);
+  grid_dep_wait();
+  // the combine kernel (or the next decode) may be scheduled now; it waits for this grid to finish
+  grid_dep_launch();
 
   if (warp == kDecConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -921,7 +961,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + ticket - 1;
         if (ticket <= 0 || item >= p.nitems) break;
         const ItemCoord c = item_coord(p, item);
-        const int raw = k == 0 ? raw_first : __ldg(p.seqlens + c.b);
+        const int raw = __ldg(p.seqlens + c.b);
         const int len = valid_len(raw + p.len_add, p.S_max);
         if (c.g == 0 && c.split == 0 && c.hsl == 0) {
           if (p.len_add ? (raw < 0 || raw >= p.S_max) : (len != raw)) {
@@ -944,6 +984,13 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           const int rows = min(kDecTileKeys, t_end - t0);
           if (it >= C::kStages) ok = mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1);
           if (!ok) break;
+#ifdef GQA_WAIT_TEST
+          // The wait-test build of the library (never the product): the first
+          // CTA issues nothing for its first item's second tile, so the stage's
+          // full barrier never completes and the consumers' bounded wait on it
+          // runs out. No load is in flight for that stage when they give up.
+          if (blockIdx.x == 0 && k == 0 && tt == 1) continue;
+#endif
           const int new_row = (p.len_add && t0 <= len - 1 && len - 1 < t0 + rows) ? len - 1 - t0 : -1;
           info[s] = StageInfo{item, rows,
                               (tt == 0 ? kTileFirst : 0) | (tt == ntiles - 1 ? kTileLast : 0) |
@@ -1165,7 +1212,10 @@ __global__ void __launch_bounds__(NT) decode_combine_kernel(OutT* __restrict__ o
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int col = tid % RL, slot = tid / RL;
   OutT* orow = out + (size_t)bh * D + slice * (D / CS);
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The next kernel on the stream (the next decode call) may be scheduled now:
+  // it only warms L2 until its own grid dependency, which includes this grid.
+  grid_dep_launch();
+  grid_dep_wait();
   if (ns == 0) {  // empty sequence
     for (int i = tid; i < D / CS; i += NT) store_out<OutT>(orow + i, 0.f);
     return;

@@ -31,6 +31,12 @@ constexpr int kWideKeys = 128;    // keys per tile: the M of S^T and the K of O^
 constexpr int kWideThreads = 192;
 constexpr int kWideTmemCols = 512;
 constexpr int kWideBox = 64;      // TMA box height of full tiles (the tail uses kDecBoxRows)
+// Keys of the first work item warmed in L2 before the grid dependency: with
+// one item per SM (long single sequences) that is the whole item.
+#ifndef GQA_WIDE_WARM_KEYS
+#define GQA_WIDE_WARM_KEYS 1024
+#endif
+constexpr int kWideWarmKeys = GQA_WIDE_WARM_KEYS;
 
 struct WideCfg {  // head dim 128
   static constexpr int D = 128;
@@ -253,17 +259,20 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023u) {
+    grid_dep_wait();
     if (threadIdx.x == 0) raise_error(GQA_DEVERR_TIMEOUT);
     return;
   }
-  // the producer fetches its first item's length before the set-up below,
-  // which hides the load's latency
-  int raw_first = 0;
+  // Launched as a programmatic dependent (as the narrow-group kernel): until
+  // grid_dep_wait() returns only the set-up below, the descriptor prefetch
+  // and an L2 warm-up of the first item's key rows (contiguous cache) run,
+  // the latter sized by a length that may be stale.
+  int spec_first = 0;
   if (warp == 4 && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k64);
     prefetch_tensormap(&tm_v64);
-    if ((int)blockIdx.x < p.nitems) raw_first = __ldg(p.seqlens + item_coord_n(p, blockIdx.x, kWideHeads).b);
+    if ((int)blockIdx.x < p.nitems) spec_first = __ldcg(p.seqlens + item_coord_n(p, blockIdx.x, kWideHeads).b);
   }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -290,7 +299,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (!kPaged && warp == 4 && lane == 0 && (int)blockIdx.x < p.nitems)
+    warm_first_item<WideCfg::D * 2>(p, item_coord_n(p, blockIdx.x, kWideHeads), spec_first, kWideWarmKeys);
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -306,7 +318,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         const int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + ticket - 1;
         if (ticket <= 0 || item >= p.nitems) break;
         const ItemCoord c = item_coord_n(p, item, kWideHeads);
-        const int raw = k == 0 ? raw_first : __ldg(p.seqlens + c.b);
+        const int raw = __ldg(p.seqlens + c.b);
         const int len = valid_len(raw + p.len_add, p.S_max);
         if (c.g == 0 && c.split == 0 && c.hsl == 0 && !p.len_add && len != raw) raise_error(GQA_DEVERR_SEQLEN);
         const int t_begin = c.split * p.chunk;

@@ -31,21 +31,44 @@ constexpr int kMaxDevices = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A runtime query that may fail (no GPU in the process) leaves its error as
+// the thread's last CUDA error. It is cleared only if no error was pending
+// before the query, so a caller's own pending error is never swallowed.
+struct QueryErrorScope {
+  const cudaError_t before = cudaPeekAtLastError();
+  void clear_own() const {
+    if (before == cudaSuccess) cudaGetLastError();
+  }
+};
+
 int current_device() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  const QueryErrorScope scope;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    scope.clear_own();
+    return -1;
+  }
   return dev;
 }
 
+// Per-device values computed once. Host threads may plan launches at the
+// same time: the entries are atomics (0 = not yet known), and two threads
+// that both compute one store the same value.
+using DeviceCache = std::atomic<int>[kMaxDevices];
+
 int sm_count(int dev) {
-  static int cache[kMaxDevices] = {0};
+  static DeviceCache cache{};
   if (dev < 0 || dev >= kMaxDevices) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
+  int n = cache[dev].load(std::memory_order_acquire);
+  if (n == 0) {
+    const QueryErrorScope scope;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      scope.clear_own();
+      n = 148;
+    }
+    cache[dev].store(n, std::memory_order_release);
   }
-  return cache[dev];
+  return n;
 }
 
 // cuTensorMapEncodeTiled from the driver, found through the runtime so the
@@ -108,7 +131,6 @@ bool encode_scales(CUtensorMap* map, const float* base, uint64_t units, uint64_t
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int launch_status() { return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA; }
 
 // ----------------------------------------------------------------------------
 // decode launch plan
@@ -166,11 +188,12 @@ bool valid_paged(const PagedCache& pc, int B, int K) {
 // Resident persistent decode CTAs per SM for head dim D (2 on B200), cached per device.
 template <int D>
 int decode_ctas_per_sm(int dev) {
-  static int cache[kMaxDevices] = {0};
+  static DeviceCache cache{};
   if (dev < 0 || dev >= kMaxDevices) return 2;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_acquire);
+  if (n == 0) {
     using C = gqa::DecCfg<D>;
+    const QueryErrorScope scope;
     if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<D, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(gqa::decode_bf16_kernel<D, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -178,40 +201,42 @@ int decode_ctas_per_sm(int dev) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_bf16_kernel<D, false, false>, gqa::kDecThreads,
                                                       C::kSmemBytes) != cudaSuccess ||
         n <= 0) {
-      cudaGetLastError();  // no GPU here: plan with the B200 figure
+      scope.clear_own();  // no GPU here: plan with the B200 figure
       n = 2;
     }
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_release);
   }
-  return cache[dev];
+  return n;
 }
 
 // Resident 8-bit-cache decode CTAs per SM (2 on B200), cached per device.
 int decode_i8_ctas_per_sm(int dev) {
-  static int cache[kMaxDevices] = {0};
+  static DeviceCache cache{};
   if (dev < 0 || dev >= kMaxDevices) return 2;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_acquire);
+  if (n == 0) {
     using C = gqa::DecCfg<128, true>;
+    const QueryErrorScope scope;
     if (cudaFuncSetAttribute(gqa::decode_bf16_kernel<128, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_bf16_kernel<128, false, true>,
                                                       gqa::kDecThreads, C::kSmemBytes) != cudaSuccess ||
         n <= 0) {
-      cudaGetLastError();
+      scope.clear_own();
       n = 2;
     }
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_release);
   }
-  return cache[dev];
+  return n;
 }
 
 // Resident wide-group decode CTAs per SM (1 on B200), cached per device.
 int wide_ctas_per_sm(int dev) {
-  static int cache[kMaxDevices] = {0};
+  static DeviceCache cache{};
   if (dev < 0 || dev >= kMaxDevices) return 1;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_acquire);
+  if (n == 0) {
+    const QueryErrorScope scope;
     if (cudaFuncSetAttribute(gqa::decode_wide_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gqa::WideCfg::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(gqa::decode_wide_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -219,12 +244,12 @@ int wide_ctas_per_sm(int dev) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa::decode_wide_kernel<false>, gqa::kWideThreads,
                                                       gqa::WideCfg::kSmemBytes) != cudaSuccess ||
         n <= 0) {
-      cudaGetLastError();
+      scope.clear_own();
       n = 1;
     }
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_release);
   }
-  return cache[dev];
+  return n;
 }
 
 // int8: the 8-bit cache (narrow-group kernel only).
@@ -295,13 +320,12 @@ int launch_decode_bf16(const DecodePlan& pl, const DecodeParams& p, const void* 
   using C = gqa::DecCfg<D>;
   decode_ctas_per_sm<D>(current_device());  // sets the shared-memory attribute once per device
   // (the scale maps of the 8-bit kernel are unused here: the K maps stand in)
+  // a programmatic dependent launch: see decode_bf16_kernel on what it does before the grid dependency
   if (p.block_table)
-    gqa::decode_bf16_kernel<D, true, false><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(
-        tk64, tv64, tk, tv, tk64, tv64, p);
-  else
-    gqa::decode_bf16_kernel<D, false, false><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(
-        tk64, tv64, tk, tv, tk64, tv64, p);
-  return launch_status();
+    return gqa::launch_kernel(gqa::decode_bf16_kernel<D, true, false>, (unsigned)pl.grid, gqa::kDecThreads,
+                              C::kSmemBytes, st, true, tk64, tv64, tk, tv, tk64, tv64, p);
+  return gqa::launch_kernel(gqa::decode_bf16_kernel<D, false, false>, (unsigned)pl.grid, gqa::kDecThreads,
+                            C::kSmemBytes, st, true, tk64, tv64, tk, tv, tk64, tv64, p);
 }
 
 // The 8-bit cache: codes [units * S_max, 128] int8, scales [units, S_max] float.
@@ -315,9 +339,8 @@ int launch_decode_i8(const DecodePlan& pl, const DecodeParams& p, const void* kc
     return GQA_ERR_CUDA;
   using C = gqa::DecCfg<128, true>;
   decode_i8_ctas_per_sm(current_device());  // sets the shared-memory attribute once per device
-  gqa::decode_bf16_kernel<128, false, true><<<(unsigned)pl.grid, gqa::kDecThreads, C::kSmemBytes, st>>>(
-      tk64, tv64, tk, tv, tks, tvs, p);
-  return launch_status();
+  return gqa::launch_kernel(gqa::decode_bf16_kernel<128, false, true>, (unsigned)pl.grid, gqa::kDecThreads,
+                            C::kSmemBytes, st, true, tk64, tv64, tk, tv, tks, tvs, p);
 }
 
 int launch_decode_wide(const DecodePlan& pl, const DecodeParams& p, const void* q, const void* kc, const void* vc,
@@ -330,20 +353,17 @@ int launch_decode_wide(const DecodePlan& pl, const DecodeParams& p, const void* 
     return GQA_ERR_CUDA;
   wide_ctas_per_sm(current_device());  // sets the shared-memory attribute once per device
   if (p.block_table)
-    gqa::decode_wide_kernel<true><<<(unsigned)pl.grid, gqa::kWideThreads, gqa::WideCfg::kSmemBytes, st>>>(
-        tq, tk64, tv64, tk16, tv16, p);
-  else
-    gqa::decode_wide_kernel<false><<<(unsigned)pl.grid, gqa::kWideThreads, gqa::WideCfg::kSmemBytes, st>>>(
-        tq, tk64, tv64, tk16, tv16, p);
-  return launch_status();
+    return gqa::launch_kernel(gqa::decode_wide_kernel<true>, (unsigned)pl.grid, gqa::kWideThreads,
+                              gqa::WideCfg::kSmemBytes, st, true, tq, tk64, tv64, tk16, tv16, p);
+  return gqa::launch_kernel(gqa::decode_wide_kernel<false>, (unsigned)pl.grid, gqa::kWideThreads,
+                            gqa::WideCfg::kSmemBytes, st, true, tq, tk64, tv64, tk16, tv16, p);
 }
 
 template <int D>
 int launch_decode_f32(const DecodePlan& pl, const DecodeParams& p, const void* kc, const void* vc,
                       cudaStream_t st) {
-  gqa::decode_f32_kernel<D><<<(unsigned)pl.grid, gqa::kDecF32Threads, 0, st>>>(
-      static_cast<const float*>(kc), static_cast<const float*>(vc), p);
-  return launch_status();
+  return gqa::launch_kernel(gqa::decode_f32_kernel<D>, (unsigned)pl.grid, gqa::kDecF32Threads, 0, st, false,
+                            static_cast<const float*>(kc), static_cast<const float*>(vc), p);
 }
 
 int launch_prefill(void* out, const void* q, const void* k, const void* v, void* k_cache, void* v_cache, int B, int S,
@@ -367,10 +387,9 @@ int launch_prefill(void* out, const void* q, const void* k, const void* v, void*
   if (rc != GQA_OK || !k_cache) return rc;
   const int cpr = d * 2 / 16;
   const long long work = 2ll * B * S * K * cpr;
-  gqa::kv_write_prompt_kernel<<<grid_for(work, 256, sms), 256, 0, st>>>(
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
-      static_cast<const uint4*>(v), B, S, K, S_max, cpr);
-  return launch_status();
+  return gqa::launch_kernel(gqa::kv_write_prompt_kernel, (unsigned)grid_for(work, 256, sms), 256, 0, st, false,
+                            static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
+                            static_cast<const uint4*>(v), B, S, K, S_max, cpr);
 }
 
 // Varlen: packed [T, heads, d] tokens of B sequences given by cu_seqlens.
@@ -384,10 +403,10 @@ int launch_prefill_varlen(void* out, const void* q, const void* k, const void* v
   if (rc != GQA_OK || !k_cache) return rc;
   const int cpr = d * 2 / 16;
   const long long work = 2ll * T * K * cpr;
-  gqa::kv_write_prompt_varlen_kernel<<<grid_for(work, 256, sms), 256, 0, st>>>(
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
-      static_cast<const uint4*>(v), cu_seqlens, B, T, K, S_max, cpr);
-  return launch_status();
+  return gqa::launch_kernel(gqa::kv_write_prompt_varlen_kernel, (unsigned)grid_for(work, 256, sms), 256, 0, st,
+                            false, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                            static_cast<const uint4*>(k), static_cast<const uint4*>(v), cu_seqlens, B, T, K, S_max,
+                            cpr);
 }
 
 // Fused K/V projection: d_model is split over CTAs (powers of two, at least
@@ -430,42 +449,35 @@ int launch_proj_d(const ProjPlan& pl, gqa::ProjParams p, const void* x, const vo
   if (!encode_rows_bf16(&tx, x, (uint64_t)p.M, (uint64_t)d_model, gqa::kPjBM) ||
       !encode_rows_bf16(&tw, w, (uint64_t)p.K * C::kN, (uint64_t)d_model, C::kN))
     return GQA_ERR_CUDA;
-  static bool configured[kMaxDevices] = {false};
+  static DeviceCache configured{};
   const int dev = current_device();
-  if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
+  if (dev >= 0 && dev < kMaxDevices && configured[dev].load(std::memory_order_acquire) == 0) {
     if (cudaFuncSetAttribute(gqa::kv_proj_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
             cudaSuccess ||
         cudaFuncSetAttribute(gqa::kv_proj_small_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gqa::PsCfg::kSmemBytes) != cudaSuccess)
       return GQA_ERR_CUDA;
-    configured[dev] = true;
+    configured[dev].store(1, std::memory_order_release);
   }
   if (pl.small) {
     CUtensorMap tx16, tw128;
     if (!encode_rows_bf16(&tx16, x, (uint64_t)p.M, (uint64_t)d_model, gqa::kPsTok) ||
         !encode_rows_bf16(&tw128, w, (uint64_t)p.K * C::kN, (uint64_t)d_model, gqa::kPsRows))
       return GQA_ERR_CUDA;
-    gqa::kv_proj_small_kernel<D><<<(unsigned)pl.grid, gqa::kPjThreads, gqa::PsCfg::kSmemBytes, st>>>(tx16, tw128, p);
+    const int rc = gqa::launch_kernel(gqa::kv_proj_small_kernel<D>, (unsigned)pl.grid, gqa::kPjThreads,
+                                      gqa::PsCfg::kSmemBytes, st, false, tx16, tw128, p);
+    if (rc != GQA_OK) return rc;
   } else {
-    gqa::kv_proj_kernel<D><<<(unsigned)pl.grid, gqa::kPjThreads, C::kSmemBytes, st>>>(tx, tw, p);
+    const int rc =
+        gqa::launch_kernel(gqa::kv_proj_kernel<D>, (unsigned)pl.grid, gqa::kPjThreads, C::kSmemBytes, st, false, tx, tw, p);
+    if (rc != GQA_OK) return rc;
   }
   if (pl.splits > 1) {  // as a programmatic dependent launch: its launch overlaps the GEMM
     const long long work = (long long)p.M * p.K * C::kN;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid_for(work, 256, sms));
-    cfg.blockDim = dim3(256);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gqa::kv_proj_finalize_kernel<D>, p) != cudaSuccess) {
-      cudaGetLastError();
-      return GQA_ERR_CUDA;
-    }
+    return gqa::launch_kernel(gqa::kv_proj_finalize_kernel<D>, (unsigned)grid_for(work, 256, sms), 256, 0, st, true,
+                              p);
   }
-  return launch_status();
+  return GQA_OK;
 }
 
 }  // namespace
@@ -505,27 +517,18 @@ size_t gqa_decode_workspace_bytes(int B, int H, int K, int S_max, int d, int num
 namespace {
 
 template <typename OutT, int D, int NT, int CS>
-cudaError_t launch_combine_t(void* out, const DecodeParams& p, const int32_t* seqlens, int H, int K, int S_max, int G,
-                             int chunk, int nsplit, int skip_single, long long units, cudaStream_t st) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(units * CS));
-  cfg.blockDim = dim3(NT);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gqa::decode_combine_kernel<OutT, D, NT, CS>, static_cast<OutT*>(out),
-                            (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, p.len_add, H, K, S_max, G, chunk,
-                            nsplit, skip_single);
+int launch_combine_t(void* out, const DecodeParams& p, const int32_t* seqlens, int H, int K, int S_max, int G,
+                     int chunk, int nsplit, int skip_single, long long units, cudaStream_t st) {
+  return gqa::launch_kernel(gqa::decode_combine_kernel<OutT, D, NT, CS>, (unsigned)(units * CS), NT, 0, st, true,
+                            static_cast<OutT*>(out), (const float*)p.ws_o, (const float2*)p.ws_ml, seqlens, p.len_add,
+                            H, K, S_max, G, chunk, nsplit, skip_single);
 }
 
 // Few splits: one CTA of 128 threads per (b, h). Many splits: four CTAs of
 // 256 threads per (b, h), a quarter of the columns each, so that more SMs
 // share the partial rows and all of them are loaded in one round.
 template <typename OutT, int D>
-cudaError_t launch_combine_d(void* out, const DecodeParams& p, const int32_t* seqlens, int H, int K, int S_max, int G,
+int launch_combine_d(void* out, const DecodeParams& p, const int32_t* seqlens, int H, int K, int S_max, int G,
                              int chunk, int nsplit, int skip_single, bool many, long long units, cudaStream_t st) {
   return many ? launch_combine_t<OutT, D, 256, 4>(out, p, seqlens, H, K, S_max, G, chunk, nsplit, skip_single, units,
                                                   st)
@@ -533,7 +536,7 @@ cudaError_t launch_combine_d(void* out, const DecodeParams& p, const int32_t* se
                                                   st);
 }
 
-cudaError_t launch_combine(void* out, const DecodeParams& p, const int32_t* seqlens, int H, int K, int S_max, int G,
+int launch_combine(void* out, const DecodeParams& p, const int32_t* seqlens, int H, int K, int S_max, int G,
                            int chunk, int nsplit, int skip_single, int d, gqa_dtype dt, bool many, long long units,
                            cudaStream_t st) {
   if (dt == GQA_BF16)
@@ -561,11 +564,11 @@ int kv_append_impl(void* k_cache, void* v_cache, const void* k_new, const void* 
   const long long work = 2ll * B * K * cpr;
   const int dev = current_device();
   const int grid = grid_for(work, 256, sm_count(dev));
-  gqa::kv_append_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k_new),
-      static_cast<const uint4*>(v_new), pos, B, K, S_max, cpr, pc ? pc->table : nullptr, pc ? pc->max_blocks : 0,
-      pc ? pc->block_size : 0, pc ? pc->num_blocks : 0);
-  return launch_status();
+  return gqa::launch_kernel(gqa::kv_append_kernel, (unsigned)grid, 256, 0, (cudaStream_t)stream, false,
+                            static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                            static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), pos, B, K, S_max, cpr,
+                            pc ? pc->table : nullptr, pc ? pc->max_blocks : 0, pc ? pc->block_size : 0,
+                            pc ? pc->num_blocks : 0);
 }
 
 // gqa_decode, and with append != 0 gqa_decode_append (seqlens then holds pos);
@@ -650,13 +653,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   // overlaps the decode kernel, and it waits for that grid before reading
   const int skip_single = dtype == GQA_BF16 ? 1 : 0;  // bf16 units with one split are already written
   const bool many = pl.nsplit > 32;
-  cudaError_t e = launch_combine(out, p, seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single, d, dtype, many,
-                                 (long long)B * H, st);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return GQA_ERR_CUDA;
-  }
-  return launch_status();
+  return launch_combine(out, p, seqlens, H, K, S_max, G, pl.chunk, pl.nsplit, skip_single, d, dtype, many,
+                        (long long)B * H, st);
 }
 
 }  // namespace
@@ -749,10 +747,9 @@ int gqa_kv_append_int8(int8_t* k_codes, float* k_scales, int8_t* v_codes, float*
   const long long warps = 2ll * B * K;
   const int dev = current_device();
   const int grid = grid_for(warps * 32, 256, sm_count(dev));
-  gqa::kv_append_int8_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
-      k_codes, k_scales, v_codes, v_scales, static_cast<const __nv_bfloat16*>(k_new),
-      static_cast<const __nv_bfloat16*>(v_new), pos, B, K, S_max);
-  return launch_status();
+  return gqa::launch_kernel(gqa::kv_append_int8_kernel, (unsigned)grid, 256, 0, (cudaStream_t)stream, false, k_codes,
+                            k_scales, v_codes, v_scales, static_cast<const __nv_bfloat16*>(k_new),
+                            static_cast<const __nv_bfloat16*>(v_new), pos, B, K, S_max);
 }
 
 size_t gqa_kv_project_workspace_bytes(int B, int T, int K, int d, int d_model) {
@@ -851,25 +848,21 @@ int gqa_meanpool_kv(void* dst, const void* src, int64_t outer, int H, int K, int
   if (inner % vec == 0 && aligned16(dst) && aligned16(src)) {
     const long long work = outer * K * (inner / vec);
     const int grid = grid_for(work, 256, sms);
-    if (dtype == GQA_BF16)
-      gqa::meanpool_vec_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-          static_cast<uint4*>(dst), static_cast<const uint4*>(src), outer, H, K, inner / vec);
-    else
-      gqa::meanpool_vec_kernel<float><<<grid, 256, 0, st>>>(static_cast<uint4*>(dst),
-                                                            static_cast<const uint4*>(src), outer, H, K, inner / vec);
+    return gqa::launch_kernel(dtype == GQA_BF16 ? gqa::meanpool_vec_kernel<__nv_bfloat16> : gqa::meanpool_vec_kernel<float>,
+                              (unsigned)grid, 256, 0, st, false, static_cast<uint4*>(dst), static_cast<const uint4*>(src),
+                              outer, H, K, inner / vec);
   } else {
     if ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & (uintptr_t)(elt - 1))
       return GQA_ERR_ALIGN;
     const long long work = outer * K * inner;
     const int grid = grid_for(work, 256, sms);
     if (dtype == GQA_BF16)
-      gqa::meanpool_scalar_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-          static_cast<__nv_bfloat16*>(dst), static_cast<const __nv_bfloat16*>(src), outer, H, K, inner);
-    else
-      gqa::meanpool_scalar_kernel<float><<<grid, 256, 0, st>>>(static_cast<float*>(dst),
-                                                               static_cast<const float*>(src), outer, H, K, inner);
+      return gqa::launch_kernel(gqa::meanpool_scalar_kernel<__nv_bfloat16>, (unsigned)grid, 256, 0, st, false,
+                                static_cast<__nv_bfloat16*>(dst), static_cast<const __nv_bfloat16*>(src), outer, H, K,
+                                inner);
+    return gqa::launch_kernel(gqa::meanpool_scalar_kernel<float>, (unsigned)grid, 256, 0, st, false,
+                              static_cast<float*>(dst), static_cast<const float*>(src), outer, H, K, inner);
   }
-  return launch_status();
 }
 
 int gqa_get_last_error(gqa_stream_t stream, uint32_t* bits) {

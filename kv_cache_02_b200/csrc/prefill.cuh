@@ -22,6 +22,8 @@
 // scheduled first.
 #pragma once
 
+#include <atomic>
+
 #include "common.cuh"
 #include "tcgen05.cuh"
 
@@ -450,14 +452,15 @@ int launch_prefill_d(PfEncodeFn fn, void* out, const void* q, const void* k, con
   if (!encode_bsh(fn, &tq, q, rows, H, D, kPfBM) || !encode_bsh(fn, &tk, k, rows, K, D, kPfBN) ||
       !encode_bsh(fn, &tv, v, rows, K, D, kPfBN))
     return GQA_ERR_CUDA;
-  static bool configured[64] = {false};
+  // once per device; concurrent host threads may both set it (same value)
+  static std::atomic<int> configured[64]{};
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+  if (dev >= 0 && dev < 64 && configured[dev].load(std::memory_order_acquire) == 0) {
     if (cudaFuncSetAttribute(prefill_causal_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
       return GQA_ERR_CUDA;
-    configured[dev] = true;
+    configured[dev].store(1, std::memory_order_release);
   }
   PrefillParams p;
   p.out = out;
@@ -471,8 +474,7 @@ int launch_prefill_d(PfEncodeFn fn, void* out, const void* q, const void* k, con
   p.cu_seqlens = cu_seqlens;
   p.T = T;
   const long long grid = cu_seqlens ? ((long long)(T + kPfBM - 1) / kPfBM + B) * H : (long long)p.n_qt * B * H;
-  prefill_causal_kernel<D><<<(unsigned)grid, kPfThreads, C::kSmemBytes, st>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+  return launch_kernel(prefill_causal_kernel<D>, (unsigned)grid, kPfThreads, C::kSmemBytes, st, false, tq, tk, tv, p);
 }
 
 }  // namespace gqa
