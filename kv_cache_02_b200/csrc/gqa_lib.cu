@@ -21,6 +21,7 @@
 #include "decode.cuh"
 #include "decode_wide.cuh"
 #include "prefill.cuh"
+#include "prefill_pair.cuh"
 #include "kv_proj.cuh"
 
 namespace {
@@ -382,6 +383,12 @@ int launch_prefill(void* out, const void* q, const void* k, const void* v, void*
   auto fn = reinterpret_cast<gqa::PfEncodeFn>(encode_fn());
   if (!fn) return GQA_ERR_CUDA;
   if ((long long)B * S >= (1ll << 31)) return GQA_ERR_SHAPE;
+  if (k_cache && (long long)B * K * S_max >= (1ll << 31)) return GQA_ERR_SHAPE;  // TMA row coordinate
+  if ((H / K) % 2 == 0)  // two heads of a group per work unit; the cache write is fused
+    return d == 128 ? gqa::launch_prefill_pair_d<128>(fn, out, q, k, v, k_cache, v_cache, B, S, H, K, S_max, scale,
+                                                      st, sms)
+                    : gqa::launch_prefill_pair_d<64>(fn, out, q, k, v, k_cache, v_cache, B, S, H, K, S_max, scale, st,
+                                                     sms);
   int rc = d == 128 ? gqa::launch_prefill_d<128>(fn, out, q, k, v, B, S, H, K, scale, st)
                     : gqa::launch_prefill_d<64>(fn, out, q, k, v, B, S, H, K, scale, st);
   if (rc != GQA_OK || !k_cache) return rc;
@@ -398,6 +405,12 @@ int launch_prefill_varlen(void* out, const void* q, const void* k, const void* v
                           cudaStream_t st, int sms) {
   auto fn = reinterpret_cast<gqa::PfEncodeFn>(encode_fn());
   if (!fn) return GQA_ERR_CUDA;
+  if (k_cache && (long long)B * K * S_max >= (1ll << 31)) return GQA_ERR_SHAPE;  // TMA row coordinate
+  if ((H / K) % 2 == 0)
+    return d == 128 ? gqa::launch_prefill_pair_d<128>(fn, out, q, k, v, k_cache, v_cache, B, 0, H, K, S_max, scale,
+                                                      st, sms, cu_seqlens, T)
+                    : gqa::launch_prefill_pair_d<64>(fn, out, q, k, v, k_cache, v_cache, B, 0, H, K, S_max, scale, st,
+                                                     sms, cu_seqlens, T);
   int rc = d == 128 ? gqa::launch_prefill_d<128>(fn, out, q, k, v, B, 0, H, K, scale, st, cu_seqlens, T)
                     : gqa::launch_prefill_d<64>(fn, out, q, k, v, B, 0, H, K, scale, st, cu_seqlens, T);
   if (rc != GQA_OK || !k_cache) return rc;
@@ -418,20 +431,61 @@ struct ProjPlan {
   size_t ws_bytes = 0;
 };
 
-// small: at most 16 tokens, the operand-swapped kernel (W_KV rows as M);
-// it fits three CTAs per SM, so it aims at two per SM.
+// small: at most 16 tokens (a decode step), the weight-streaming GEMV: one
+// CTA per 16 W_KV rows over all of d_model, no split, no workspace.
+// Otherwise the token-tile GEMM, d_model split while tiles leave SMs idle.
 ProjPlan plan_proj(long long M, int K, int d, int d_model, int sms) {
   ProjPlan pl;
-  const int ksteps = d_model / gqa::kPjBK;
   pl.small = M <= gqa::kPsTok;
-  const long long base = pl.small ? (long long)K * 2 * d / gqa::kPsRows : (M + gqa::kPjBM - 1) / gqa::kPjBM * K;
-  const long long target = pl.small ? 2ll * sms : sms;
-  while (base * pl.splits < target && ksteps % (pl.splits * 2) == 0 && ksteps / (pl.splits * 2) >= 4 &&
+  if (pl.small) {
+    pl.grid = (long long)K * 2 * d / gqa::kGvRows;
+    return pl;
+  }
+  const int ksteps = d_model / gqa::kPjBK;
+  const long long base = (M + gqa::kPjBM - 1) / gqa::kPjBM * K;
+  while (base * pl.splits < sms && ksteps % (pl.splits * 2) == 0 && ksteps / (pl.splits * 2) >= 4 &&
          pl.splits * 2 <= gqa::kPjMaxSplits)
     pl.splits *= 2;
   pl.grid = base * pl.splits;
   pl.ws_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)M * K * 2 * d * sizeof(float) : 0;
   return pl;
+}
+
+// A 3-D bf16 view of a row-major [rows, cols] matrix as (64 columns, rows,
+// cols / 64 blocks of 64 columns), box (64, box_rows, box_blocks), 128-byte
+// swizzle: one load brings box_rows rows x 64 box_blocks columns, block-major.
+bool encode_row_blocks_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                            uint32_t box_blocks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {cols * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_blocks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int NT>
+int launch_proj_gemv(const ProjPlan& pl, const gqa::ProjParams& p, const void* x, const void* w, int d_model,
+                     cudaStream_t st) {
+  using G = gqa::GvCfg<NT>;
+  CUtensorMap tx, tw;
+  if (!encode_row_blocks_bf16(&tx, x, (uint64_t)p.M, (uint64_t)d_model, 8 * NT, gqa::kGvCols / 64) ||
+      !encode_row_blocks_bf16(&tw, w, (uint64_t)p.K * 2 * D, (uint64_t)d_model, gqa::kGvRows, gqa::kGvCols / 64))
+    return GQA_ERR_CUDA;
+  static DeviceCache configured{};
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxDevices && configured[dev].load(std::memory_order_acquire) == 0) {
+    if (cudaFuncSetAttribute(gqa::kv_proj_gemv_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             G::kSmemBytes) != cudaSuccess)
+      return GQA_ERR_CUDA;
+    configured[dev].store(1, std::memory_order_release);
+  }
+  // a programmatic dependent launch: it warms L2 with its W_KV rows before the grid dependency
+  return gqa::launch_kernel(gqa::kv_proj_gemv_kernel<D, NT>, (unsigned)pl.grid, G::kThreads, G::kSmemBytes, st, true,
+                            tx, tw, p, d_model);
 }
 
 bool valid_proj(int B, int T, int K, int S_max, int d, int d_model) {
@@ -445,6 +499,8 @@ template <int D>
 int launch_proj_d(const ProjPlan& pl, gqa::ProjParams p, const void* x, const void* w, int d_model, cudaStream_t st,
                   int sms) {
   using C = gqa::PjCfg<D>;
+  if (pl.small)
+    return p.M <= 8 ? launch_proj_gemv<D, 1>(pl, p, x, w, d_model, st) : launch_proj_gemv<D, 2>(pl, p, x, w, d_model, st);
   CUtensorMap tx, tw;
   if (!encode_rows_bf16(&tx, x, (uint64_t)p.M, (uint64_t)d_model, gqa::kPjBM) ||
       !encode_rows_bf16(&tw, w, (uint64_t)p.K * C::kN, (uint64_t)d_model, C::kN))
@@ -453,21 +509,11 @@ int launch_proj_d(const ProjPlan& pl, gqa::ProjParams p, const void* x, const vo
   const int dev = current_device();
   if (dev >= 0 && dev < kMaxDevices && configured[dev].load(std::memory_order_acquire) == 0) {
     if (cudaFuncSetAttribute(gqa::kv_proj_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(gqa::kv_proj_small_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gqa::PsCfg::kSmemBytes) != cudaSuccess)
+        cudaSuccess)
       return GQA_ERR_CUDA;
     configured[dev].store(1, std::memory_order_release);
   }
-  if (pl.small) {
-    CUtensorMap tx16, tw128;
-    if (!encode_rows_bf16(&tx16, x, (uint64_t)p.M, (uint64_t)d_model, gqa::kPsTok) ||
-        !encode_rows_bf16(&tw128, w, (uint64_t)p.K * C::kN, (uint64_t)d_model, gqa::kPsRows))
-      return GQA_ERR_CUDA;
-    const int rc = gqa::launch_kernel(gqa::kv_proj_small_kernel<D>, (unsigned)pl.grid, gqa::kPjThreads,
-                                      gqa::PsCfg::kSmemBytes, st, false, tx16, tw128, p);
-    if (rc != GQA_OK) return rc;
-  } else {
+  {
     const int rc =
         gqa::launch_kernel(gqa::kv_proj_kernel<D>, (unsigned)pl.grid, gqa::kPjThreads, C::kSmemBytes, st, false, tx, tw, p);
     if (rc != GQA_OK) return rc;
@@ -774,6 +820,7 @@ int gqa_kv_project_append(void* k_cache, void* v_cache, const void* x, const voi
   gqa::ProjParams p;
   p.k_cache = k_cache;
   p.v_cache = v_cache;
+  p.w = w_kv;
   p.pos = pos;
   p.ws = static_cast<float*>(workspace);
   p.B = B;

@@ -17,7 +17,7 @@
 // split over CTAs: each split writes its fp32 partial tile to a workspace
 // slice of its own (no atomics, nothing to zero) and kv_proj_finalize_kernel
 // sums the splits and writes the rows. A decode step (a few tokens) uses
-// kv_proj_small_kernel, with the operands swapped.
+// kv_proj_gemv_kernel, which streams W_KV once with no split.
 #pragma once
 
 #include "common.cuh"
@@ -45,6 +45,7 @@ struct PjCfg {
 struct ProjParams {
   void* k_cache;         // [B, K, S_max, D] bf16
   void* v_cache;
+  const void* w;         // W_KV [K * 2D, d_model] bf16 (for the L2 warm-up of a decode step)
   const int32_t* pos;    // [B]: key of each sequence's first new token, or null (0)
   float* ws;             // splits > 1: partials [splits][M][K * 2D] fp32
   int B, T, K, S_max, M, ksteps_per_split, splits;
@@ -187,132 +188,177 @@ __global__ void __launch_bounds__(kPjThreads, 1)
   }
 }
 
-// A decode step (at most kPsTok tokens): the operands swap. A = 128 rows of
-// W_KV (outputs), B = the tokens (padded to 16), D = [128 outputs x 16
-// tokens] in TMEM (lane = output), so the MMA does 16x less padding work
-// than with tokens as M and every CTA streams its own slice of W_KV.
-// Epilogue thread r holds output r for every token: across a warp 32
-// consecutive outputs of one token, 64 contiguous bytes of a cache row.
-constexpr int kPsRows = 128;  // W_KV rows (outputs) per CTA
-constexpr int kPsTok = 16;    // tokens (MMA N)
+// A decode step (at most kPsTok = 16 tokens): a weight-streaming GEMV.
+// Every W_KV row is read once and multiplied by the few tokens: 2 * tokens
+// flop per 2 bytes of W, so HBM bound; the tensor cores are needed only to
+// keep up with the stream (fp32 FMA would not), and the warp-level
+// mma.sync m16n8k16 fits a 16-row x 8-token tile without padding rows.
+//
+// One CTA owns 16 consecutive W_KV rows (outputs) over all of d_model, so
+// there is no split and nothing to merge across CTAs: no workspace and no
+// second pass. Its W slice streams through a ring of kGvStages stages of 512
+// columns (16 KB of W with the same columns of x) loaded by TMA; with
+// d_model = 4096 the whole 128 KB slice is requested at once. Consumer warp
+// w takes the stages w, w + kGvStages, ...: per 16 columns an ldmatrix of W
+// (A, 16 rows), an ldmatrix of x (B, 8 tokens) per 8 tokens, one MMA. At the
+// end the warps' partial tiles are summed in shared memory and the rows
+// written, bf16, at each token's key.
+constexpr int kPsTok = 16;    // most tokens of a decode step
+constexpr int kGvRows = 16;   // W_KV rows per CTA
+constexpr int kGvCols = 512;  // d_model columns per stage (8 blocks of 64)
+#ifndef GQA_GV_WARM
+#define GQA_GV_WARM 1
+#endif
+constexpr bool kGvWarm = GQA_GV_WARM != 0;  // L2 warm-up of the W_KV slice before the grid dependency
 
-struct PsCfg {
-  static constexpr int kABytes = kPsRows * kPjBK * 2;  // 16 KB of W
-  static constexpr int kBBytes = kPsTok * kPjBK * 2;   // 2 KB of x
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBarOff = kPjStages * kStageBytes;
-  static constexpr int kNumBars = 2 * kPjStages + 1;
-  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
-  static constexpr int kTmemCols = 32;  // 16 used (the allocation minimum is 32)
+template <int NT>  // token tiles of 8: 1 (up to 8 tokens) or 2 (up to 16)
+struct GvCfg {
+  static constexpr int kStages = NT == 1 ? 8 : 6;          // = consumer warps
+  static constexpr int kThreads = (kStages + 1) * 32;      // + the TMA producer warp
+  static constexpr int kWBytes = kGvRows * kGvCols * 2;    // 16 KB
+  static constexpr int kXBytes = 8 * NT * kGvCols * 2;     // 8 KB per token tile
+  static constexpr int kStageBytes = kWBytes + kXBytes;
+  static constexpr int kRedOff = kStages * kStageBytes;    // [warps][16 rows][8 NT tokens] fp32
+  static constexpr int kBarOff = kRedOff + kStages * kGvRows * 8 * NT * 4;
+  static constexpr int kSmemBytes = kBarOff + 2 * kStages * 8;
 };
 
-template <int D>
-__global__ void __launch_bounds__(kPjThreads)
-    kv_proj_small_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                         const ProjParams p) {
-  using C = PsCfg;
+// tm_w: W_KV as (64 columns, rows, d_model / 64 blocks), box (64, 16, 8);
+// tm_x: x as (64, tokens, d_model / 64), box (64, 8 NT, 8) (token rows past
+// the batch read as zeros). Both 128-byte swizzled: in a stage, W block b,
+// row r is the 128-byte line b * 16 + r, x block b, token n the line b * 8 NT + n.
+template <int D, int NT>
+__global__ void __launch_bounds__(GvCfg<NT>::kThreads, 1)
+    kv_proj_gemv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                        const ProjParams p, int d_model) {
+  using C = GvCfg<NT>;
+  constexpr int kW = C::kStages;  // consumer warps
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kPjStages;
-  uint64_t* acc_full = empty + kPjStages;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  float* red = reinterpret_cast<float*>(smem + C::kRedOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* empty = full + kW;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nkb = (d_model + kGvCols - 1) / kGvCols;  // stages of the whole row slice
+  const int row0 = (int)blockIdx.x * kGvRows;
 
   if (smem_u32(smem) & 1023u) {
+    grid_dep_wait();
     if (threadIdx.x == 0) raise_error(GQA_DEVERR_TIMEOUT);
     return;
   }
-  const int ft = (int)(blockIdx.x / p.splits);  // tile of 128 W_KV rows
-  const int sp = (int)(blockIdx.x % p.splits);
-  const int k_begin = sp * p.ksteps_per_split;
-  const int nk = p.ksteps_per_split;
-
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPjStages; ++s) {
+    for (int s = 0; s < kW; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
     fence_mbar_init();
   }
-  if (warp == 5) {
-    tmem_alloc(tmem_holder, C::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the finalize pass may be scheduled
+  // W_KV rows are weights: warm L2 with this CTA's slice while the kernel
+  // before finishes (a hint; the loads below come after the grid dependency)
+  if (kGvWarm && warp == kW && lane < kGvRows)
+    for (int c = 0; c < d_model * 2; c += 32768)
+      prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(p.w) + ((size_t)(row0 + lane) * d_model) * 2 + c,
+                       (uint32_t)min(32768, d_model * 2 - c));
+  grid_dep_wait();
+  grid_dep_launch();
 
-  if (warp == 4) {
+  if (warp == kW) {
+    // ------------------------------------------------------------ producer
+    // The first pass over the ring is issued by one lane per stage at once;
+    // stages past it (d_model > kW * 512) by lane 0 as consumers free them.
+    const uint64_t pol_w = l2_policy_evict_first();  // streamed once
+    const uint64_t pol_x = l2_policy_evict_last();   // read by every CTA
+    auto issue = [&](int j) {
+      const int s = j % kW;
+      uint8_t* st = smem + s * C::kStageBytes;
+      mbar_arrive_expect_tx(&full[s], (uint32_t)C::kStageBytes);
+      tma_load_3d(st, &tm_w, 0, row0, j * (kGvCols / 64), &full[s], pol_w);
+      tma_load_3d(st + C::kWBytes, &tm_x, 0, 0, j * (kGvCols / 64), &full[s], pol_x);
+    };
     if (lane == 0) {
-      prefetch_tensormap(&tm_x);
       prefetch_tensormap(&tm_w);
-      const uint64_t pol_x = l2_policy_evict_last();
-      const uint64_t pol_w = l2_policy_evict_first();
-      int issued = 0;
-      for (int j = 0; j < nk; ++j) {
-        const int s = j % kPjStages;
-        if (j >= kPjStages && !mbar_wait_bounded(&empty[s], ((j / kPjStages) - 1) & 1)) break;
-        uint8_t* st = smem + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)C::kStageBytes);
-        const int kx = (k_begin + j) * kPjBK;
-        tma_load_2d(st, &tm_w, kx, ft * kPsRows, &full[s], pol_w);
-        tma_load_2d(st + C::kABytes, &tm_x, kx, 0, &full[s], pol_x);
+      prefetch_tensormap(&tm_x);
+    }
+    __syncwarp();
+    if (lane < min(kW, nkb)) issue(lane);
+    if (lane == 0) {
+      int issued = min(kW, nkb);
+      for (int j = kW; j < nkb; ++j) {
+        if (!mbar_wait_bounded(&empty[j % kW], ((j / kW) - 1) & 1)) break;
+        issue(j);
         ++issued;
       }
-      for (int j = max(0, issued - kPjStages); j < issued; ++j) mbar_wait_bounded(&full[j % kPjStages], (j / kPjStages) & 1);
+      // this CTA's loads land before it may exit (the consumers may have given up)
+      for (int j = max(0, issued - kW); j < issued; ++j) mbar_wait_bounded(&full[j % kW], (j / kW) & 1);
     }
-  } else if (warp == 5) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kPsRows, kPsTok, false, false);
-      bool ok = true;
-      for (int j = 0; j < nk && ok; ++j) {
-        const int s = j % kPjStages;
-        if (!(ok = mbar_wait_bounded(&full[s], (j / kPjStages) & 1))) break;
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * C::kStageBytes);
-        const uint32_t b_addr = a_addr + C::kABytes;
-#pragma unroll
-        for (int kk = 0; kk < kPjBK / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-          tc_mma(tmem, ad, bd, idesc, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&empty[s]);
-      }
-      tc_commit(acc_full);
-    }
-  } else {
-    const int f = ft * kPsRows + threadIdx.x;  // W_KV row: head f / 2D, K (< D) or V, dim f % D
-    const int g = f / (2 * D), jd = f % (2 * D);
-    if (__all_sync(0xffffffffu, mbar_wait_bounded(acc_full, 0))) {
-      tc_fence_after();
-      float o[16];
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), o);
-      tc_wait_ld();
-      const size_t ncols = (size_t)p.K * 2 * D;
-#pragma unroll
-      for (int t = 0; t < kPsTok; ++t) {
-        if (t >= p.M) break;
-        if (p.splits > 1) {
-          p.ws[((size_t)sp * p.M + t) * ncols + f] = o[t];
-        } else {
-          size_t row = 0;
-          if (!proj_row(p, t, g, row)) continue;
-          __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(jd < D ? p.k_cache : p.v_cache);
-          cache[row * D + (jd % D)] = __float2bfloat16_rn(o[t]);
-        }
-      }
-    }
+    return;
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 5) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+
+  // -------------------------------------------------------------- consumers
+  // ldmatrix rows: A (W) matrices (rows 0-7 | 8-15) x (chunk c | c+1); B (x)
+  // matrices (tokens 0-7) x (chunks c, c+1, c+2, c+3): two 16-column steps
+  const int a_row = (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int a_chk = lane >> 4;
+  const int b_tok = lane & 7;
+  const int b_chk = lane >> 3;
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  bool ok = true;
+  for (int j = warp, n = 0; j < nkb; j += kW, ++n) {
+    if (!(ok = mbar_wait_bounded(&full[warp], n & 1))) break;
+    const uint32_t wa = smem_u32(smem + warp * C::kStageBytes);
+    const uint32_t xa = wa + C::kWBytes;
+#pragma unroll 4
+    for (int b = 0; b < kGvCols / 64; ++b) {  // 64-column block: 4 steps of 16 columns
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {           // two steps at a time: chunks 4h .. 4h + 3
+        uint32_t a[2][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int line = b * kGvRows + a_row;
+          const int chk = 4 * h + 2 * u + a_chk;
+          ldmatrix_x4(wa + line * 128 + ((chk ^ (line & 7)) << 4), a[u][0], a[u][1], a[u][2], a[u][3]);
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const int line = b * 8 * NT + 8 * t + b_tok;
+          const int chk = 4 * h + b_chk;
+          uint32_t x0, x1, x2, x3;
+          ldmatrix_x4(xa + line * 128 + ((chk ^ (line & 7)) << 4), x0, x1, x2, x3);
+          mma_bf16_16816(acc[t], a[0][0], a[0][1], a[0][2], a[0][3], x0, x1);
+          mma_bf16_16816(acc[t], a[1][0], a[1][1], a[1][2], a[1][3], x2, x3);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[warp]);
+  }
+  // the warps' partial [16 rows x 8 NT tokens] tiles: accumulator (row g | g + 8, tokens 2c, 2c + 1)
+  const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    float* rw = red + (size_t)warp * kGvRows * 8 * NT;
+    rw[g * 8 * NT + 8 * t + 2 * c] = acc[t][0];
+    rw[g * 8 * NT + 8 * t + 2 * c + 1] = acc[t][1];
+    rw[(g + 8) * 8 * NT + 8 * t + 2 * c] = acc[t][2];
+    rw[(g + 8) * 8 * NT + 8 * t + 2 * c + 1] = acc[t][3];
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kW * 32) : "memory");  // the consumer warps (the producer has left)
+  // output (row r, token m): thread m * 16 + r, 16 rows of a token = 32 contiguous bytes of a cache row
+  for (int o = threadIdx.x; o < kGvRows * 8 * NT; o += kW * 32) {
+    const int m = o / kGvRows, r = o % kGvRows;
+    if (m >= p.M) continue;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kW; ++w) sum += red[((size_t)w * kGvRows + r) * 8 * NT + m];
+    const int f = row0 + r;  // W_KV row: head f / 2D, K (< D) or V, dim f % D
+    const int gh = f / (2 * D), jd = f % (2 * D);
+    size_t crow = 0;
+    if (!proj_row(p, m, gh, crow)) continue;
+    __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(jd < D ? p.k_cache : p.v_cache);
+    cache[crow * D + (jd % D)] = __float2bfloat16_rn(sum);
   }
 }
 

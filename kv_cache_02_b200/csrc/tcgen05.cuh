@@ -98,6 +98,17 @@ __device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const float (
       : "memory");
 }
 
+// True in one lane of the (converged) warp, false in the others.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Shared-memory matrix descriptor (sm100): 128-byte swizzle, version 1.

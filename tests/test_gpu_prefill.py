@@ -49,6 +49,9 @@ SMALL = [
     (2, 517, 12, 4, 128),   # G = 3
     (1, 64, 2, 2, 64),      # a single key tile
     (1, 1, 4, 2, 128),      # one token
+    (4, 1024, 32, 8, 128),  # 512 head-pair units: several per persistent CTA
+    (2, 1500, 16, 2, 64),   # G = 8 (four head pairs), d = 64, ragged, several units per CTA
+    (1, 700, 16, 4, 128),   # ragged: a last key tile of 60 rows
 ]
 
 
@@ -65,14 +68,20 @@ def test_prefill_small_full_compare(gqa, shape):
         assert np.array_equal(got[:, 0, h], inp["v"][:, 0, h // (H // K)])
 
 
-def test_prefill_writes_the_cache(gqa):
-    B, S, H, K, d, S_max = 2, 200, 8, 2, 128, 333
-    inp = make(B, S, H, K, d, 0x9F77)
-    _, kc, vc = run(gqa, inp, 0.1, S_max=S_max)
+@pytest.mark.parametrize("shape", [(2, 200, 8, 2, 128, 333), (1, 300, 4, 2, 64, 300), (2, 1024, 16, 4, 128, 1100),
+                                   (2, 300, 12, 4, 128, 320)],
+                         ids=["G4_tail72", "G2_d64_full", "G4_many_units", "G3_separate_write"])
+def test_prefill_writes_the_cache(gqa, shape):
+    # even G: the prefill kernel stores each key tile from shared memory (TMA
+    # for whole 16-row groups, plain stores for the rest); odd G: a separate pass
+    B, S, H, K, d, S_max = shape
+    inp = make(B, S, H, K, d, 0x9F77 + S)
+    got, kc, vc = run(gqa, inp, 0.1, S_max=S_max)
     want_k, want_v = oracle.prefill_cache_write(inp["k"], inp["v"], S_max,
                                                 np.full((B, K, S_max, d), 0x7FC0, np.uint16),
                                                 np.full((B, K, S_max, d), 0x7FC0, np.uint16))
     assert np.array_equal(kc, want_k) and np.array_equal(vc, want_v)
+    assert_close(got, oracle.prefill_causal(inp["q"], inp["k"], inp["v"], 0.1), str(shape))
 
 
 def test_prefill_large_scores_stay_finite(gqa):

@@ -43,8 +43,11 @@ def run(gqa, x, w, S_max, pos):
 
 CASES = [
     # B, T, K, d, d_model, S_max, pos
-    (8, 1, 8, 128, 4096, 64, (63, 0, 5, 17, 30, 40, 50, 60)),  # a decode step: d_model split
+    (8, 1, 8, 128, 4096, 64, (63, 0, 5, 17, 30, 40, 50, 60)),  # a decode step: the weight-streaming GEMV
     (3, 1, 2, 64, 512, 16, (0, 15, 7)),                         # d = 64
+    (4, 4, 8, 128, 8192, 64, (0, 60, 33, 7)),                   # 16 tokens (two token tiles), the ring reused
+    (2, 3, 4, 64, 1088, 32, (3, 29)),                           # a last stage of 64 columns
+    (1, 1, 1, 64, 8192, 8, (7,)),                               # 128 W_KV rows: 8 CTAs, ring reused
     (2, 300, 4, 128, 1024, 320, (0, 20)),                        # a prompt: 300 tokens (ragged tiles)
     (1, 129, 1, 128, 256, 129, None),                            # MQA, pos None (0)
 ]

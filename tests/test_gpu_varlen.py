@@ -53,6 +53,7 @@ CASES = [
     ((1000, 33), 4, 4, 64),                # MHA, d = 64
     ((200, 200, 200), 12, 4, 128),         # equal lengths, G = 3
     (tuple(int(x) for x in np.random.default_rng(5).integers(0, 150, 40)), 4, 2, 64),  # 40 short prompts
+    ((900, 1100, 37, 640, 1500), 32, 8, 128),  # 560 head-pair units: several per persistent CTA
 ]
 
 
