@@ -492,10 +492,12 @@ def small_kernel_measurements(args, peaks, steps, only=None):
                 if it >= args.warmup:
                     t[with_cache].append(a.elapsed_time(b))
         ms = statistics.median(t[True]) - statistics.median(t[False])
-        byts = 2 * 2 * w.B * w.S * w.K * w.d * 2  # K and V read once and written once
-        gbs = byts / (ms * 1e-3) / 1e9 if ms > 0 else None
-        res[PROMPT_WRITE] = {"ms": round(ms, 5), "bytes": byts, "GB/s": None if gbs is None else round(gbs, 1),
-                             "frac_of_measured_hbm": None if gbs is None else round(gbs / peaks["hbm_gbs"], 4),
+        byts = w.B * w.S * w.K * w.d * 2 * 2  # the K and V rows written to the caches
+        res[PROMPT_WRITE] = {"increment_ms": round(ms, 5), "bytes_written": byts,
+                             "with_write_ms": round(statistics.median(t[True]), 5),
+                             "without_write_ms": round(statistics.median(t[False]), 5),
+                             "how": "the prefill stores each key tile to the cache from shared memory while it "
+                                    "computes (no separate pass); the increment is what the stores cost it",
                              "timing": "gqa_prefill_causal with the cache write less without it, medians, "
                                        "each call after an L2 flush"}
         del q, k, v, out, kc, vc, flush
@@ -777,6 +779,16 @@ def proj_measurement(args, name, peaks, steps):
          "GB/s": round(byts / (ms * 1e-3) / 1e9, 1), "l2": "flushed (512 MiB write, then 512 MiB read)"}
     if M < 512:
         r["frac_of_measured_hbm"] = round(r["GB/s"] / peaks["hbm_gbs"], 4)
+        # a decode step's projection also back to back, over rotating W_KV copies (>= 2x L2 of distinct
+        # weights), as the calls of a model's layers run: no L2 flush kernel between the calls
+        def make_call(i):
+            wi = to_dev(inp["w_kv"])
+            return lambda: gqa.gqa_kv_project_append(kc, vc, x, wi, pos, ws)
+
+        bms = back_to_back_ms(make_call, N * w.d_model * 2, steps)
+        bgbs = byts / (bms * 1e-3) / 1e9
+        r["back_to_back"] = {"ms": round(bms, 5), "GB/s": round(bgbs, 1),
+                             "frac_of_measured_hbm": round(bgbs / peaks["hbm_gbs"], 4), "timing": BACK_TO_BACK}
     else:
         r["frac_of_measured_bf16_burst"] = round(r["TFLOP/s"] / peaks["bf16_tflops"], 4)
     del x, wk, pos, kc, vc, ws, flush

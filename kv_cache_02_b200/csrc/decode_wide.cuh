@@ -391,44 +391,58 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     }
   } else if (warp == 5) {
     // -------------------------------------------------------------- MMA
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(kWideHeads, kWideKeys, false, false);  // Q K^T
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kWideHeads, D, false, true);          // P V, V MN-major
-      const uint32_t q_addr = smem_u32(smem + C::kQOff);
-      const uint32_t p_addr = smem_u32(smem + C::kPOff);
-      int nitem = 0;  // items started
-      int prev_first = 0, prev_ord = 0;  // tile j-1: opened its item; ordinal of its item
-      int cur_ord = 0;
-      bool ok = true;
-      int j = 0;
-      auto issue_pv = [&](int t, int first, int ord) -> bool {
-        if (!mbar_wait_bounded(p_full, t & 1)) return false;
-        // the first PV of an item overwrites O^T: the previous item's epilogue must have read it
-        if (first && ord >= 1 && !mbar_wait_bounded(o_free, (ord - 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(smem + C::kKVOff + (t % C::kStages) * C::kStage + C::kTile);
+    // The warp runs converged (descriptors are warp-uniform values) and one
+    // elected lane issues each tcgen05 instruction: issued from a single-lane
+    // branch, each MMA paid for moving its operands to uniform registers.
+    const bool leader = elect_one();
+    constexpr uint32_t idesc_s = idesc_bf16_f32(kWideHeads, kWideKeys, false, false);  // Q K^T
+    constexpr uint32_t idesc_o = idesc_bf16_f32(kWideHeads, D, false, true);          // P V, V MN-major
+    const uint32_t q_addr = smem_u32(smem + C::kQOff);
+    const uint32_t p_addr = smem_u32(smem + C::kPOff);
+    int nitem = 0;  // items started
+    int prev_first = 0, prev_ord = 0;  // tile j-1: opened its item; ordinal of its item
+    int cur_ord = 0;
+    bool ok = true;
+    int j = 0;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (leader) tc_commit(bar);
+      __syncwarp();
+    };
+    auto issue_pv = [&](int t, int first, int ord) -> bool {
+      if (!wait_all(p_full, t & 1)) return false;
+      // the first PV of an item overwrites O^T: the previous item's epilogue must have read it
+      if (first && ord >= 1 && !wait_all(o_free, (ord - 1) & 1)) return false;
+      tc_fence_after();
+      const uint32_t v_addr = smem_u32(smem + C::kKVOff + (t % C::kStages) * C::kStage + C::kTile);
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < kWideKeys / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * C::kPHalf + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, C::kHalf, 1024);
           tc_mma(tmem + C::kOCol, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
         }
-        tc_commit(pv_done);
-        tc_commit(&kv_empty[t % C::kStages]);
-        return true;
-      };
-      for (;; ++j) {
-        const int s = j % C::kStages;
-        if (!(ok = mbar_wait_bounded(&kv_full[s], (j / C::kStages) & 1))) break;
-        const StageInfo si = info[s];
-        if (si.item < 0) break;
-        if (si.flags & kTileFirst) {
-          if (!(ok = mbar_wait_bounded(q_full, nitem & 1))) break;
-          cur_ord = nitem++;
-        }
-        if (j >= 2 && !(ok = mbar_wait_bounded(&s_free[j & 1], ((j >> 1) - 1) & 1))) break;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + C::kKVOff + s * C::kStage);
+      }
+      __syncwarp();
+      commit(pv_done);
+      commit(&kv_empty[t % C::kStages]);
+      return true;
+    };
+    for (;; ++j) {
+      const int s = j % C::kStages;
+      if (!(ok = wait_all(&kv_full[s], (j / C::kStages) & 1))) break;
+      const StageInfo si = info[s];
+      if (si.item < 0) break;
+      if (si.flags & kTileFirst) {
+        if (!(ok = wait_all(q_full, nitem & 1))) break;
+        cur_ord = nitem++;
+      }
+      if (j >= 2 && !(ok = wait_all(&s_free[j & 1], ((j >> 1) - 1) & 1))) break;
+      tc_fence_after();
+      const uint32_t k_addr = smem_u32(smem + C::kKVOff + s * C::kStage);
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk & 3) * 32;
@@ -436,16 +450,17 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           const uint64_t bd = smem_desc_sw128(k_addr + (kk >> 2) * C::kHalf + off, 16, 1024);
           tc_mma(tmem + C::kSCol + (uint32_t)((j & 1) * kWideKeys), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&s_full[j & 1]);
-        if (si.flags & kTileLast) tc_commit(q_empty);  // the item's last S: Q may be replaced
-        if (j >= 1 && !(ok = issue_pv(j - 1, prev_first, prev_ord))) break;
-        prev_first = si.flags & kTileFirst;
-        prev_ord = cur_ord;
       }
-      if (ok && j >= 1) issue_pv(j - 1, prev_first, prev_ord);
-      tc_commit(mma_done);  // completes when every MMA issued above has finished
-      mbar_wait_bounded(mma_done, 0);
+      __syncwarp();
+      commit(&s_full[j & 1]);
+      if (si.flags & kTileLast) commit(q_empty);  // the item's last S: Q may be replaced
+      if (j >= 1 && !(ok = issue_pv(j - 1, prev_first, prev_ord))) break;
+      prev_first = si.flags & kTileFirst;
+      prev_ord = cur_ord;
     }
+    if (ok && j >= 1) issue_pv(j - 1, prev_first, prev_ord);
+    commit(mma_done);  // completes when every MMA issued above has finished
+    wait_all(mma_done, 0);
   } else {
     // ---------------------------------------------------- softmax / epilogue
     // warp w serves heads 16 w .. 16 w + 15 (TMEM lanes 32 w .. 32 w + 15):

@@ -130,15 +130,17 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     }
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kPjBM, C::kN, false, false);
-      bool ok = true;
-      for (int j = 0; j < nk && ok; ++j) {
-        const int s = j % kPjStages;
-        if (!(ok = mbar_wait_bounded(&full[s], (j / kPjStages) & 1))) break;
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * C::kStageBytes);
-        const uint32_t b_addr = a_addr + C::kABytes;
+    // converged warp (warp-uniform descriptors), one elected lane issues
+    const bool leader = elect_one();
+    constexpr uint32_t idesc = idesc_bf16_f32(kPjBM, C::kN, false, false);
+    bool ok = true;
+    for (int j = 0; j < nk && ok; ++j) {
+      const int s = j % kPjStages;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (j / kPjStages) & 1)))) break;
+      tc_fence_after();
+      const uint32_t a_addr = smem_u32(smem + s * C::kStageBytes);
+      const uint32_t b_addr = a_addr + C::kABytes;
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < kPjBK / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
@@ -147,8 +149,10 @@ __global__ void __launch_bounds__(kPjThreads, 1)
         }
         tc_commit(&empty[s]);
       }
-      tc_commit(acc_full);  // completes when every MMA issued above has finished
+      __syncwarp();
     }
+    if (leader) tc_commit(acc_full);  // completes when every MMA issued above has finished
+    __syncwarp();
   } else {
     // ----------------------------------------------------------- epilogue
     const int r = threadIdx.x;  // token row within the tile = TMEM lane

@@ -247,18 +247,28 @@ __global__ void __launch_bounds__(kPfThreads, 2)
     }
   } else if (warp == 5) {
     // -------------------------------------------------------------- MMA
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(kPfBM, kPfBN, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kPfBM, D, false, true);
-      const uint32_t q_addr = smem_u32(smem + C::kQOff);
-      const uint32_t p_addr = smem_u32(smem + C::kPOff);
-      bool ok = mbar_wait_bounded(q_full, 0);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % kPfStages;
-        if (!mbar_wait_bounded(&k_full[s], (j / kPfStages) & 1)) return false;
-        if (j >= 2 && !mbar_wait_bounded(&s_free[j & 1], ((j >> 1) - 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + C::kKVOff + s * C::kStageBytes);
+    // The warp runs converged (descriptors are warp-uniform values) and one
+    // elected lane issues each tcgen05 instruction.
+    const bool leader = elect_one();
+    constexpr uint32_t idesc_s = idesc_bf16_f32(kPfBM, kPfBN, false, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(kPfBM, D, false, true);
+    const uint32_t q_addr = smem_u32(smem + C::kQOff);
+    const uint32_t p_addr = smem_u32(smem + C::kPOff);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (leader) tc_commit(bar);
+      __syncwarp();
+    };
+    bool ok = wait_all(q_full, 0);
+    auto issue_s = [&](int j) -> bool {
+      const int s = j % kPfStages;
+      if (!wait_all(&k_full[s], (j / kPfStages) & 1)) return false;
+      if (j >= 2 && !wait_all(&s_free[j & 1], ((j >> 1) - 1) & 1)) return false;
+      tc_fence_after();
+      const uint32_t k_addr = smem_u32(smem + C::kKVOff + s * C::kStageBytes);
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk & 3) * 32;  // 16 columns = 32 bytes inside the 128-byte swizzle row
@@ -266,34 +276,38 @@ __global__ void __launch_bounds__(kPfThreads, 2)
           const uint64_t bd = smem_desc_sw128(k_addr + (kk >> 2) * C::kKVHalf + off, 16, 1024);
           tc_mma(tmem + (uint32_t)((j & 1) * kPfBN), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&s_full[j & 1]);
-        tc_commit(&k_empty[s]);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_s(j + 1)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait_bounded(p_full, j & 1) || !mbar_wait_bounded(&v_full[j % kPfStages], (j / kPfStages) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(smem + C::kKVOff + (j % kPfStages) * C::kStageBytes + C::kTileBytes);
+      }
+      __syncwarp();
+      commit(&s_full[j & 1]);
+      commit(&k_empty[s]);
+      return true;
+    };
+    if (ok) ok = issue_s(0);
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      if (j + 1 < n_tiles && !issue_s(j + 1)) {
+        ok = false;
+        break;
+      }
+      if (!wait_all(p_full, j & 1) || !wait_all(&v_full[j % kPfStages], (j / kPfStages) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t v_addr = smem_u32(smem + C::kKVOff + (j % kPfStages) * C::kStageBytes + C::kTileBytes);
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < kPfBN / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(p_addr + kk * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(v_addr + kk * 16 * 128, C::kKVHalf, 1024);
           tc_mma(tmem + C::kOCol, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(pv_done);
-        tc_commit(&v_empty[j % kPfStages]);
       }
-      tc_commit(mma_done);
-      mbar_wait_bounded(mma_done, 0);
+      __syncwarp();
+      commit(pv_done);
+      commit(&v_empty[j % kPfStages]);
     }
+    commit(mma_done);
+    wait_all(mma_done, 0);
   } else {
     // ---------------------------------------------------------- softmax
     const int r = threadIdx.x;  // query row within the tile = TMEM lane

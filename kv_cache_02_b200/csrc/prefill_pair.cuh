@@ -11,21 +11,26 @@
 // i + 2 grid, ... of a list ordered sequence by sequence, each sequence's
 // heaviest (latest) query tiles first.
 //
-// Warp roles (10 warps):
-//   warps 0-3  softmax of tile 0: thread r owns query row r (TMEM lane r)
-//   warps 4-7  softmax of tile 1
-//   warp 8     TMEM allocation; one thread issues every tcgen05.mma
-//   warp 9     TMA loads: lane 0 the K tiles, lane 1 the V tiles, lane 2 the
+// Warp roles (18 warps):
+//   warps 8 t + 4 h + q (t, h in {0, 1}, q = 0..3): the softmax of tile t
+//              for keys 64 h .. 64 h + 63 of each 128-key tile; thread q 32 +
+//              lane owns query row q 32 + lane (TMEM lane). The two warps
+//              with the same t and q hold the same rows (partner warps) and
+//              exchange row maxima, checks and sums through shared memory
+//              with a 64-thread named barrier.
+//   warp 16    TMEM allocation; the converged warp issues every tcgen05.mma
+//              from one elected lane
+//   warp 17    TMA loads: lane 0 the K tiles, lane 1 the V tiles, lane 2 the
 //              Q tiles (128 keys per K/V tile, two stages each); the owner of
 //              a key tile also stores it to the KV cache from shared memory
 // TMEM (512 columns): S_t at columns 128 t (fp32, 128 keys) and O_t at
-// 256 + 128 t (fp32, D columns). The softmax writes P_t (bf16 pairs) over
-// the upper 64 columns of S_t, and P_t V is issued with A read from TMEM, so
-// P never goes through shared memory.
+// 256 + 128 t (fp32, D columns). Each softmax half writes its P (bf16 pairs)
+// over the first 32 of its own 64 score columns, and P_t V is issued with A
+// read from TMEM, so P never goes through shared memory.
 //
 // The chain of a tile from one softmax step to the next is kept short:
-//   * P_t(j) V is issued in two halves, the first (keys 0-63) as soon as the
-//     softmax has stored that half of P;
+//   * P_t(j) V is issued in two halves, each as soon as the softmax warps
+//     of that key half have stored their P;
 //   * S_t(j+1) follows the second half (it overwrites P_t(j)), and its
 //     completion hands it to the softmax;
 //   * the softmax computes the exponentials against the running maximum
@@ -52,9 +57,9 @@ namespace gqa {
 constexpr int kPpBM = 128;      // query rows per tile
 constexpr int kPpBN = 128;      // keys per K/V tile and per S tile
 constexpr int kPpStages = 2;    // K and V ring stages
-constexpr int kPpThreads = 320;
+constexpr int kPpThreads = 576;
 constexpr int kPpTmemCols = 512;
-constexpr int kPpMmaWarp = 8;
+constexpr int kPpMmaWarp = 16;
 // Every kPpPolyEvery-th pair of exponentials is computed on the FMA pipe
 // (exp2_poly2), the rest by the MUFU unit; 0: all by the MUFU unit.
 #ifndef GQA_PP_POLY_EVERY
@@ -74,7 +79,7 @@ __device__ __forceinline__ bool pp_wait(uint64_t* bar, uint32_t parity) {
   if constexpr (GQA_PP_SLEEP_NS > 0) return mbar_wait_bounded_sleep(bar, parity, GQA_PP_SLEEP_NS);
   return mbar_wait_bounded(bar, parity);
 }
-constexpr int kPpLoadWarp = 9;
+constexpr int kPpLoadWarp = 17;
 
 template <int D>
 struct PpCfg {
@@ -86,10 +91,11 @@ struct PpCfg {
   static constexpr int kQOff = 0;                                 // Q0, Q1
   static constexpr int kKOff = kQOff + 2 * kQBytes;               // K stages
   static constexpr int kVOff = kKOff + kPpStages * kKVBytes;      // V stages
-  static constexpr int kBarOff = kVOff + kPpStages * kKVBytes;
+  static constexpr int kXOff = kVOff + kPpStages * kKVBytes;  // partner exchange [2 tiles][2 slots][2 halves][128]
+  static constexpr int kBarOff = kXOff + 2 * 2 * 2 * kPpBM * 4;
   // q_full[2] q_empty[2] k_full[S] k_empty[S] v_full[S] v_empty[S] s_full[2] p_lo[2] p_hi[2] o_ready[2]
-  // o_free[2] mma_done
-  static constexpr int kNumBars = 4 + 4 * kPpStages + 10 + 1;
+  // o_free[2] mma_done pair[8]
+  static constexpr int kNumBars = 4 + 4 * kPpStages + 10 + 1 + 8;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kOCol = 256;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -289,8 +295,9 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   uint64_t* p_lo = s_full + 2;          // [2 tiles] P_t of keys 0-63 stored (O_t rescaled): 128 arrivals
   uint64_t* p_hi = p_lo + 2;            // [2 tiles] P_t of keys 64-127 stored: 128 arrivals
   uint64_t* o_ready = p_hi + 2;         // [2 tiles] the unit's last P_t V finished
-  uint64_t* o_free = o_ready + 2;       // [2 tiles] the epilogue has read O_t: 128 arrivals
+  uint64_t* o_free = o_ready + 2;       // [2 tiles] the epilogue has read O_t: 256 arrivals
   uint64_t* mma_done = o_free + 2;      // every MMA of the CTA finished (before TMEM is released)
+  uint64_t* pair = mma_done + 1;        // [2 tiles][4 row groups] the partner warps' exchanges: 64 arrivals
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -306,7 +313,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       mbar_init(&p_lo[i], 128);
       mbar_init(&p_hi[i], 128);
       mbar_init(&o_ready[i], 1);
-      mbar_init(&o_free[i], 128);
+      mbar_init(&o_free[i], 256);
     }
     for (int i = 0; i < S; ++i) {
       mbar_init(&k_full[i], 1);
@@ -315,6 +322,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       mbar_init(&v_empty[i], 1);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&pair[i], 64);
     fence_mbar_init();
   }
   if (warp == kPpMmaWarp) {
@@ -424,13 +432,13 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       }
       __syncwarp();
     };
-    // one half (keys 64 hh ..) of O_t += P_t V, V in stage vs, P_t in columns 128 t + 64 + 32 hh
+    // one half (keys 64 hh ..) of O_t += P_t V, V in stage vs, P_t in columns 128 t + 64 hh .. + 31
     auto issue_pv_half = [&](int t, int vs, int hh, bool acc) {
       const uint64_t vd = v_desc + (uint64_t)((vs * C::kKVBytes) >> 4);
       if (leader) {
 #pragma unroll
         for (int kk = 4 * hh; kk < 4 * hh + 4; ++kk)
-          tc_mma_tmem_a(tmem + C::kOCol + (uint32_t)(t * 128), tmem + (uint32_t)(t * kPpBN + 64 + kk * 8),
+          tc_mma_tmem_a(tmem + C::kOCol + (uint32_t)(t * 128), tmem + (uint32_t)(t * kPpBN + 64 * hh + (kk - 4 * hh) * 8),
                         vd + (uint64_t)((kk * 16 * 128) >> 4), idesc_o, (acc || kk > 0) ? 1u : 0u);
       }
       __syncwarp();
@@ -486,13 +494,30 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     wait_all(mma_done, 0);
   } else {
     // ----------------------------------------------------- softmax + epilogue
-    const int t = warp >> 2;          // query tile of this warpgroup
-    const int r = threadIdx.x & 127;  // row within the tile = TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t s_addr = lane_base + (uint32_t)(t * kPpBN);
+    const int t = warp >> 3, hh = (warp >> 2) & 1, q = warp & 3;
+    const int r = q * 32 + lane;  // row within the tile = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    const uint32_t s_addr = lane_base + (uint32_t)(t * kPpBN + 64 * hh);  // this half's 64 score columns
     const uint32_t o_addr = lane_base + (uint32_t)(C::kOCol + t * 128);
+    float* xbuf = reinterpret_cast<float*>(smem + C::kXOff) + t * (2 * 2 * kPpBM);
+    uint64_t* xbar = &pair[t * 4 + q];  // the partner warps' barrier (a bounded wait, unlike bar.sync)
+    int xc = 0;                         // exchanges made (their slot and the barrier phase alternate)
+    // this row's value from the partner warp (the other key half); NaN if the partner never came.
+    // Every lane of both warps calls it (64 arrivals); it returns with the warp converged, as the
+    // warp-collective tcgen05 loads and stores that follow require.
+    auto exchange = [&](float v) -> float {
+      float* e = xbuf + (xc & 1) * (2 * kPpBM);
+      e[hh * kPpBM + r] = v;
+      mbar_arrive(xbar);
+      const bool came = pp_wait(xbar, xc & 1);
+      ++xc;
+      const float o = came ? e[(1 - hh) * kPpBM + r] : __int_as_float(0x7fc00000);
+      __syncwarp();
+      return o;
+    };
     const float sl2 = p.scale_log2;
     const bool pos_scale = sl2 > 0.f;
+    const float xs = pos_scale ? sl2 : 1.f;  // the scale still to apply to the loaded scores
     int sp = 0, units = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok; u += gridDim.x, ++units) {
@@ -500,7 +525,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       if (!pair_unit(p, u, b, seq0, len, qt, g, pr)) break;
       const int nt = qt + 1;
       const int qpos = qt * kPpBM + r;
-      float m_used = -INFINITY, l = 0.f;
+      float m_used = -INFINITY, l = 0.f;  // l: this half's share of the row sum
       for (int j = 0; j < nt; ++j, ++sp) {
         // tcgen05.ld/st are warp-collective: every decision that guards them is warp-uniform
         if (!__all_sync(0xffffffffu, pp_wait(&s_full[t], sp & 1))) {
@@ -508,68 +533,88 @@ __global__ void __launch_bounds__(kPpThreads, 1)
           break;
         }
         tc_fence_after();
-        const int kmax = min(qpos, len - 1) - j * kPpBN;  // keys j*128 + c with c <= kmax are visible
-        const float xs = pos_scale ? sl2 : 1.f;          // the scale still to apply to the loaded scores
-        float x[128];
-        // S_t into registers, masked; with a non-positive scale the scores are scaled here
-        auto load_s = [&]() {
+        // keys 64 hh + 32 c + i of the tile with i <= kmax - 32 c are visible
+        const int kmax = min(qpos, len - 1) - j * kPpBN - 64 * hh;
+        float x[32];
+        auto load_chunk = [&](int c) {
+          tmem_ld32(s_addr + 32 * c, x);
+          tc_wait_ld();
+          const int km = kmax - 32 * c;
+          if (!(pos_scale && km >= 31)) {
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + c4 * 32, *reinterpret_cast<float(*)[32]>(&x[32 * c4]));
-          tc_wait_ld();  // one wait for the four loads
-          if (!(pos_scale && kmax >= kPpBN - 1)) {
-#pragma unroll
-            for (int c = 0; c < 128; ++c) x[c] = c <= kmax ? (pos_scale ? x[c] : x[c] * sl2) : -INFINITY;
+            for (int i = 0; i < 32; ++i) x[i] = i <= km ? (pos_scale ? x[i] : x[i] * sl2) : -INFINITY;
           }
         };
-        // the row maximum of the tile (log2 units, scale applied) and the step of m_used it implies
+        // the maximum of this half of the row (log2 units, scale applied; -inf if all masked)
+        auto half_max = [&]() -> float {
+          float m = -INFINITY;
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            load_chunk(c);
+            float a = fmax3(x[0], x[1], x[2]);
+#pragma unroll
+            for (int i = 3; i < 31; i += 2) a = fmax3(a, x[i], x[i + 1]);
+            m = fmaxf(m, fmaxf(a, x[31]));
+          }
+          return m * xs;
+        };
+        uint32_t pk[32];
+        auto half_exps = [&]() -> float {
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            load_chunk(c);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float y0, y1, p0, p1;
+              fma2(y0, y1, x[2 * i], x[2 * i + 1], xs, -m_used);
+              if (kPpPolyEvery > 0 && i % (kPpPolyEvery > 0 ? kPpPolyEvery : 1) == kPpPolyEvery - 1) {  // FMA pipe
+                exp2_poly2(y0, y1, p0, p1);
+              } else {
+                p0 = fast_exp2(y0);
+                p1 = fast_exp2(y1);
+              }
+              if (i & 1)
+                add2(s2, s3, p0, p1);
+              else
+                add2(s0, s1, p0, p1);
+              pk[16 * c + i] = kPpIntPack ? pack_bf16x2_int(p0, p1) : pack_bf16x2(p0, p1);
+            }
+          }
+          return (s0 + s1) + (s2 + s3);
+        };
         float alpha = 1.f;
         bool rescale = false;
-        auto take_max = [&]() {
-          const float mt = fmaxf(max64(*reinterpret_cast<const float(*)[64]>(&x[0])),
-                                 max64(*reinterpret_cast<const float(*)[64]>(&x[64]))) * xs;
-          if (mt > m_used + 8.f) {  // first tile: m_used = -inf
-            const float m_new = fmaxf(mt, m_used);
+        // a new row maximum m_t: the running maximum moves only when m_t exceeds it by more than 8
+        auto take_max = [&](float m_t) {
+          if (m_t > m_used + 8.f) {  // first tile: m_used = -inf (its key 0 is visible to every row)
+            const float m_new = fmaxf(m_t, m_used);
             alpha = fast_exp2(m_used - m_new);
             rescale = j > 0;
             m_used = m_new;
           }
         };
-        uint32_t pk[64];
-        float tsum = 0.f;
-        auto exps = [&]() {
-          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            float y0, y1, p0, p1;
-            fma2(y0, y1, x[2 * c], x[2 * c + 1], xs, -m_used);
-            if (kPpPolyEvery > 0 && c % (kPpPolyEvery > 0 ? kPpPolyEvery : 1) == kPpPolyEvery - 1) {  // FMA pipe
-              exp2_poly2(y0, y1, p0, p1);
-            } else {
-              p0 = fast_exp2(y0);
-              p1 = fast_exp2(y1);
-            }
-            if (c & 1)
-              add2(s2, s3, p0, p1);
-            else
-              add2(s0, s1, p0, p1);
-            pk[c] = kPpIntPack ? pack_bf16x2_int(p0, p1) : pack_bf16x2(p0, p1);
-          }
-          tsum = (s0 + s1) + (s2 + s3);
-        };
-        load_s();
-        if (j == 0) take_max();
-        exps();
-        // every P of the tile is at most 2^8 when their sum is (otherwise, or
-        // on a NaN, the row maximum is taken and the tile recomputed from S)
-        if (__any_sync(0xffffffffu, !(tsum <= 256.f))) {
-          load_s();
-          take_max();
-          exps();
+        if (j == 0) {
+          const float mh = half_max();
+          take_max(fmaxf(mh, exchange(mh)));
         }
-        l = l * alpha + tsum;
-        // the P V before this tile's S has finished: O_t may be rescaled now,
-        // before the first half of P V(j) may run
-        if (__any_sync(0xffffffffu, rescale)) {
+        float sh = half_exps();
+        if (j > 0) {
+          // every P of the row is at most 2^8 when the sum of each half is;
+          // otherwise (or on a NaN) both halves take the row maximum and recompute
+          const bool fail = !(sh <= 256.f);
+          const float partner_fail = exchange(fail ? 1.f : 0.f);  // every lane exchanges, failing or not
+          const bool row_fail = fail || partner_fail != 0.f;
+          if (__any_sync(0xffffffffu, row_fail)) {  // the partner warp holds the same rows: it takes this branch too
+            const float mh = half_max();
+            take_max(fmaxf(mh, exchange(mh)));
+            sh = half_exps();
+          }
+        }
+        l = l * alpha + sh;
+        // the P V before this tile's S has finished: O_t may be rescaled now
+        // (by the first half's warps, before the first half of P V(j) may run)
+        if (hh == 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
           for (int cb = 0; cb < D; cb += 32) {
             float o[32];
@@ -580,32 +625,27 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             tmem_st32(o_addr + cb, o);
           }
         }
-        tmem_st16_u(s_addr + 64, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-        tmem_st16_u(s_addr + 80, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+        tmem_st16_u(s_addr, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+        tmem_st16_u(s_addr + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
         tc_wait_st();
         tc_fence_before();
-        mbar_arrive(&p_lo[t]);  // keys 0-63: the first half of P V may run
-        tmem_st16_u(s_addr + 96, *reinterpret_cast<const uint32_t(*)[16]>(&pk[32]));
-        tmem_st16_u(s_addr + 112, *reinterpret_cast<const uint32_t(*)[16]>(&pk[48]));
-        tc_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_hi[t]);
+        mbar_arrive(hh == 0 ? &p_lo[t] : &p_hi[t]);
       }
       if (!ok) break;
-      // epilogue: O_t / l -> bf16 rows of head g G + 2 pr + t
+      // epilogue: O_t / l -> bf16 rows of head g G + 2 pr + t, each half of the warps D / 2 columns
+      const float inv_l = 1.f / (l + exchange(l));
       if (!__all_sync(0xffffffffu, pp_wait(&o_ready[t], units & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float inv_l = 1.f / l;
       const int h = g * p.G + 2 * pr + t;
       uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                            (((size_t)seq0 + qpos) * p.H + h) * D);
+                                            (((size_t)seq0 + qpos) * p.H + h) * D + hh * (D / 2));
 #pragma unroll 1
-      for (int cb = 0; cb < D; cb += 32) {
+      for (int cb = 0; cb < D / 2; cb += 32) {
         float o[32];
-        tmem_ld32(o_addr + cb, o);
+        tmem_ld32(o_addr + hh * (D / 2) + cb, o);
         tc_wait_ld();
         if (qpos < len) {
 #pragma unroll
