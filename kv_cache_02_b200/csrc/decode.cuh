@@ -889,6 +889,29 @@ __device__ __forceinline__ void warm_first_item(const DecodeParams& p, const Ite
   }
 }
 
+// The paged form of warm_first_item, by the producer warp: lane i asks L2
+// for the rows of block i of the item's first max_keys keys (a table entry
+// read through L2 that may be stale; an entry outside the pool is skipped).
+template <int D>
+__device__ __forceinline__ void warm_first_item_paged(const DecodeParams& p, const ItemCoord& c, int raw, int max_keys,
+                                                      int lane) {
+  if (c.hsl != 0) return;
+  const int len = valid_len(raw + p.len_add, p.S_max);
+  const int t_begin = c.split * p.chunk;
+  const int t_end = min(min(len, t_begin + p.chunk), t_begin + max_keys);
+  if (t_end <= t_begin) return;
+  const int bs = p.block_size;
+  const int blk = t_begin / bs + lane;  // the lane's block of the sequence
+  if (blk * bs >= t_end) return;
+  const int e = __ldcg(p.block_table + (size_t)c.b * p.max_blocks + blk);
+  if ((unsigned)e >= (unsigned)p.num_blocks) return;
+  const int r0 = max(t_begin, blk * bs), r1 = min(t_end, (blk + 1) * bs);  // keys of the block to warm
+  const size_t off = ((size_t)(e * p.K + c.g) * bs + (r0 - blk * bs)) * D * 2;
+  const uint32_t bytes = (uint32_t)(r1 - r0) * D * 2;
+  prefetch_l2_bulk(static_cast<const uint8_t*>(p.k_cache_w) + off, bytes);
+  prefetch_l2_bulk(static_cast<const uint8_t*>(p.v_cache_w) + off, bytes);
+}
+
 // kPaged: the cache is a paged pool; kInt8: the cache holds 8-bit codes and
 // per-row scales (tm_k*/tm_v* then map codes, tm_ks/tm_vs the scales; the
 // bf16 kernels ignore tm_ks/tm_vs).
@@ -915,10 +938,11 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   }
   // Launched as a programmatic dependent: until grid_dep_wait() returns, the
   // previous kernel on the stream may still be running. Before it: the
-  // barriers, the descriptor prefetch, and (contiguous caches) an L2 warm-up
-  // of the first work item's key rows, sized by a length read that may be
-  // stale -- a hint only, so the rows may still be being written. After it
-  // the length is read again and every input is read for real.
+  // barriers, the descriptor prefetch, and an L2 warm-up of the first work
+  // item's key rows (of a paged cache through its table), sized by a length
+  // read that may be stale -- a hint only, so the rows may still be being
+  // written. After it the length is read again and every input is read for
+  // real.
   int spec_first = 0;
   if (!kPaged && warp == kDecConsumerWarps && lane == 0) {
     prefetch_tensormap(&tm_k64);
@@ -942,6 +966,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   __syncthreads();
   if (!kPaged && warp == kDecConsumerWarps && lane == 0 && (int)blockIdx.x < p.nitems)
     warm_first_item<D * C::kElt>(p, item_coord(p, blockIdx.x), spec_first, kDecWarmKeys);
+  if (kPaged && warp == kDecConsumerWarps && (int)blockIdx.x < p.nitems) {
+    const ItemCoord c0 = item_coord(p, blockIdx.x);
+    warm_first_item_paged<D>(p, c0, __ldcg(p.seqlens + c0.b), kDecWarmKeys, lane);
+  }
   grid_dep_wait();
   // the combine kernel (or the next decode) may be scheduled now; it waits for this grid to finish
   grid_dep_launch();

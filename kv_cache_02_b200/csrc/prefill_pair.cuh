@@ -61,12 +61,15 @@ constexpr int kPpThreads = 576;
 constexpr int kPpTmemCols = 512;
 constexpr int kPpMmaWarp = 16;
 // Every kPpPolyEvery-th pair of exponentials is computed on the FMA pipe
-// (exp2_poly2), the rest by the MUFU unit; 0: all by the MUFU unit.
+// (exp2_poly2), the rest by the MUFU unit; 0: all by the MUFU unit. One in
+// eight measured fastest (0.527 ms against 0.538 with none and 0.556 with one
+// in four on the 4 x 4096 x 32 x 128 prefill).
 #ifndef GQA_PP_POLY_EVERY
-#define GQA_PP_POLY_EVERY 0
+#define GQA_PP_POLY_EVERY 8
 #endif
 constexpr int kPpPolyEvery = GQA_PP_POLY_EVERY;
 // P to bf16: 0 the conversion instruction, 1 integer round-to-nearest-even, 2 integer round-half-up
+// (the integer forms move the conversion off the XU pipe; measured slower here)
 #ifndef GQA_PP_PACK
 #define GQA_PP_PACK 0
 #endif
