@@ -71,21 +71,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// try_wait with a suspend-time hint: a thread whose phase is not complete
-// sleeps (up to hint_ns) instead of returning at once, so waiting warps take
-// no issue slots from the warps that share their scheduler.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait until the phase with the given parity has completed. Returns false
 // (and raises GQA_DEVERR_TIMEOUT) if that takes longer than kWaitLimitNs
 // after the first 256 unsuccessful tries: the clock is read only every 256
@@ -95,24 +80,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
-      const unsigned long long t = globaltimer_ns();
-      if (t0 == 0) {
-        t0 = t;
-      } else if (t - t0 > kWaitLimitNs) {
-        raise_error(GQA_DEVERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-// mbar_wait_bounded with sleeping tries (mbar_try_wait_sleep): the clock is
-// read every 16 tries, each of which sleeps at most hint_ns.
-__device__ __forceinline__ bool mbar_wait_bounded_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  unsigned long long t0 = 0;
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
-    if ((it & 15u) == 0) {
       const unsigned long long t = globaltimer_ns();
       if (t0 == 0) {
         t0 = t;

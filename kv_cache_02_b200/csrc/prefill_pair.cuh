@@ -68,20 +68,7 @@ constexpr int kPpMmaWarp = 16;
 #define GQA_PP_POLY_EVERY 8
 #endif
 constexpr int kPpPolyEvery = GQA_PP_POLY_EVERY;
-// P to bf16: 0 the conversion instruction, 1 integer round-to-nearest-even, 2 integer round-half-up
-// (the integer forms move the conversion off the XU pipe; measured slower here)
-#ifndef GQA_PP_PACK
-#define GQA_PP_PACK 0
-#endif
-constexpr bool kPpIntPack = GQA_PP_PACK != 0;
-// The kernel's barrier waits sleep up to this long per try (0: plain tries)
-#ifndef GQA_PP_SLEEP_NS
-#define GQA_PP_SLEEP_NS 0
-#endif
-__device__ __forceinline__ bool pp_wait(uint64_t* bar, uint32_t parity) {
-  if constexpr (GQA_PP_SLEEP_NS > 0) return mbar_wait_bounded_sleep(bar, parity, GQA_PP_SLEEP_NS);
-  return mbar_wait_bounded(bar, parity);
-}
+__device__ __forceinline__ bool pp_wait(uint64_t* bar, uint32_t parity) { return mbar_wait_bounded(bar, parity); }
 constexpr int kPpLoadWarp = 17;
 
 template <int D>
@@ -260,22 +247,6 @@ __device__ __forceinline__ void exp2_poly2(float y0, float y1, float& e0, float&
   fma2v(p0, p1, p0, p1, f0, f1, 0.999928236f);
   e0 = y0 < -125.f ? 0.f : __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
   e1 = y1 < -125.f ? 0.f : __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
-// Two floats -> bf16 pair (lo in the low half), rounded to nearest-even
-// with integer operations: the conversion instruction would share the XU
-// pipe with the softmax's exponentials, the integer adds and the byte
-// permute do not. Inputs are finite and non-negative (probabilities).
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
-  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-#if GQA_PP_PACK == 2  // round half up (ties away from zero)
-  a += 0x8000u;
-  b += 0x8000u;
-#else                 // round to nearest-even
-  a += 0x7FFFu + ((a >> 16) & 1u);
-  b += 0x7FFFu + ((b >> 16) & 1u);
-#endif
-  return __byte_perm(a, b, 0x7632);  // the high halves: bytes 2, 3 of a, then of b
 }
 
 template <int D>
@@ -581,7 +552,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 add2(s2, s3, p0, p1);
               else
                 add2(s0, s1, p0, p1);
-              pk[16 * c + i] = kPpIntPack ? pack_bf16x2_int(p0, p1) : pack_bf16x2(p0, p1);
+              pk[16 * c + i] = pack_bf16x2(p0, p1);
             }
           }
           return (s0 + s1) + (s2 + s3);
