@@ -158,11 +158,14 @@ def test_projection_rejects_bad_arguments(lib):
     assert f(P, P, P, P, None, 2, 1, 8, 64, 96, 4096, None, 0, 1, None) == -2    # head dim
     assert f(P, P, P, P, None, 2, 1, 8, 64, 128, 4000, None, 0, 1, None) == -2   # d_model not a multiple of 64
     assert f(P, P, P, P, None, 2, 1, 8, 64, 128, 4096, None, 0, 0, None) == -6   # f32
-    assert f(P, P, P, P, None, 2, 1, 8, 64, 128, 4096, None, 0, 1, None) == -1   # needs a workspace (8 tokens)
+    # a 256-token prompt: its d_model is split over CTAs, which needs a workspace
+    assert f(P, P, P, P, None, 2, 128, 8, 1024, 128, 4096, None, 0, 1, None) == -1
     assert f(P, P, P + 2, P, None, 2, 1, 8, 64, 128, 4096, None, 0, 1, None) == -3
     assert f(None, None, None, None, None, 0, 1, 8, 64, 128, 4096, None, 0, 1, None) == 0
     ws = lib.gqa_kv_project_workspace_bytes
-    assert ws(8, 1, 8, 128, 4096) > 0 and ws(4, 4096, 8, 128, 4096) == 0 and ws(8, 1, 8, 128, 100) == 0
+    assert ws(8, 1, 8, 128, 4096) == 0       # a decode step (<= 16 tokens): the GEMV, no split
+    assert ws(2, 128, 8, 128, 4096) > 0      # a short prompt split over d_model
+    assert ws(4, 4096, 8, 128, 4096) == 0 and ws(8, 1, 8, 128, 100) == 0
 
 
 def test_prefill_rejects_bad_arguments(lib):
