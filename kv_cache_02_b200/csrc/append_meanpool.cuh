@@ -218,6 +218,21 @@ __global__ void meanpool_vec_kernel(uint4* __restrict__ dst, const uint4* __rest
     const uint4* s = src + ((o * H + (long long)g * G) * inner_vecs + iv);
     double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     int r = 0;
+    // eight source vectors requested before any is summed (the summation
+    // order stays r = 0, 1, ..., G - 1): 0.71 -> 0.76 of the copy bandwidth
+    // for 64 -> 8 heads, against four at a time
+    for (; r + 8 <= G; r += 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = __ldg(s + (long long)(r + q) * inner_vecs);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        double x[8];
+        widen16(v[q], x, (const T*)nullptr);
+#pragma unroll
+        for (int k = 0; k < N; ++k) acc[k] += x[k];
+      }
+    }
     for (; r + 4 <= G; r += 4) {
       uint4 v0 = __ldg(s + (long long)(r + 0) * inner_vecs);
       uint4 v1 = __ldg(s + (long long)(r + 1) * inner_vecs);
