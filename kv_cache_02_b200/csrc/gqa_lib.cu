@@ -272,10 +272,12 @@ DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gq
     // narrow groups: about eight small work items per SM (their partials are
     // small), twelve for bf16 batches of many units, where the finer items
     // shorten the tail (split sweeps: the 70B ragged batch 2 % faster, the
-    // Llama-3-8B layer within 1 %; the 8-bit consumers pay more per item and
-    // are slower with more); wide groups: about one item per SM, since a
-    // 64-head partial is 32 KB; never below 256 keys per split
-    const long long per_sm = (!int8 && units >= 32) ? 12 : 8;
+    // Llama-3-8B layer within 1 %), six for the 8-bit cache, whose consumers
+    // pay more per item (split sweeps: the Llama-3-8B shape 0.72 -> 0.74 of
+    // the copy bandwidth at 14 splits instead of 19, the 70B ragged batch
+    // 0.84 -> 0.87 at 4 instead of 5); wide groups: about one item per SM,
+    // since a 64-head partial is 32 KB; never below 256 keys per split
+    const long long per_sm = int8 ? 6 : (units >= 32 ? 12 : 8);
     const long long target = pl.wide ? (long long)sms : per_sm * sms;
     splits = (int)std::max<long long>(1, (target + units - 1) / std::max<long long>(units, 1));
     splits = std::min(splits, std::max(1, (S_max + 255) / 256));
