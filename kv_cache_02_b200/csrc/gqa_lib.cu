@@ -255,7 +255,7 @@ int wide_ctas_per_sm(int dev) {
 
 // int8: the 8-bit cache (narrow-group kernel only).
 DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gqa_dtype dt, int sms,
-                       bool int8 = false) {
+                       bool int8 = false, bool paged = false) {
   DecodePlan pl;
   const int G = H / K;
   pl.wide = !int8 && dt == GQA_BF16 && d == 128 && G % gqa::kWideHeads == 0;
@@ -276,11 +276,15 @@ DecodePlan plan_decode(int B, int H, int K, int S_max, int d, int num_splits, gq
     // pay more per item (split sweeps: the Llama-3-8B shape 0.72 -> 0.74 of
     // the copy bandwidth at 14 splits instead of 19, the 70B ragged batch
     // 0.84 -> 0.87 at 4 instead of 5); wide groups: about one item per SM,
-    // since a 64-head partial is 32 KB; never below 256 keys per split
+    // since a 64-head partial is 32 KB; never below 256 keys per split, nor
+    // below 448 for a paged cache, whose producer loads an item's window of
+    // the block table at its start (Llama-3-8B layer at block size 16: 0.86
+    // of the copy bandwidth with 320-key splits, 0.89 with 448)
     const long long per_sm = int8 ? 6 : (units >= 32 ? 12 : 8);
     const long long target = pl.wide ? (long long)sms : per_sm * sms;
+    const int min_chunk = paged ? 448 : 256;
     splits = (int)std::max<long long>(1, (target + units - 1) / std::max<long long>(units, 1));
-    splits = std::min(splits, std::max(1, (S_max + 255) / 256));
+    splits = std::min(splits, std::max(1, (S_max + min_chunk - 1) / min_chunk));
     splits = std::min(splits, max_splits);
   }
   int chunk = (S_max + splits - 1) / splits;
@@ -641,7 +645,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   if (append && (!k_new || !v_new)) return GQA_ERR_INVALID_ARG;
   if (append && (!aligned16(k_new) || !aligned16(v_new))) return GQA_ERR_ALIGN;
   const int dev = current_device();
-  const DecodePlan pl = plan_decode(B, H, K, S_max, d, num_splits, dtype, sm_count(dev), int8);
+  const DecodePlan pl = plan_decode(B, H, K, S_max, d, num_splits, dtype, sm_count(dev), int8, pc != nullptr);
   if (pl.ws_bytes == (size_t)-1) return GQA_ERR_SHAPE;  // more work items than the work counter holds
   if (pl.ws_bytes > 0) {
     if (!workspace || workspace_bytes < pl.ws_bytes) return GQA_ERR_INVALID_ARG;
@@ -843,7 +847,7 @@ size_t gqa_decode_paged_workspace_bytes(int B, int H, int K, int d, int block_si
     return 0;
   const int S_max = max_blocks * block_size;
   if (!valid_decode_shape(B, H, K, S_max, d, true) || num_splits < 0) return 0;
-  const DecodePlan a = plan_decode(B, H, K, S_max, d, num_splits, GQA_BF16, sm_count(current_device()));
+  const DecodePlan a = plan_decode(B, H, K, S_max, d, num_splits, GQA_BF16, sm_count(current_device()), false, true);
   if (a.ws_bytes == (size_t)-1) return 0;
   return a.ws_bytes;
 }

@@ -223,6 +223,9 @@ PAGED_WORKLOADS = {
         "paged_llama3_8b_decode_b8_h32_k8_d128_s8192_bs16", "llama3_8b_decode_b8_h32_k8_d128_s8192", 16, 64),
     "paged_ragged_70b_decode_b32_h64_k8_d128_s1k_16k_bs64": PagedShape(
         "paged_ragged_70b_decode_b32_h64_k8_d128_s1k_16k_bs64", "ragged_70b_decode_b32_h64_k8_d128_s1k_16k", 64, 64),
+    # multi-query attention (G = 64, the tensor-core wide path) over a paged 128K-token context
+    "paged_long_ctx_mqa_b1_h64_k1_d128_s131072_bs16": PagedShape(
+        "paged_long_ctx_mqa_b1_h64_k1_d128_s131072_bs16", "long_ctx_mqa_b1_h64_k1_d128_s131072", 16, 64),
 }
 
 

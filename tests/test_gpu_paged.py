@@ -86,8 +86,11 @@ def test_paged_decode_small(gqa, case, num_splits):
     assert status == (0, 0)
     ref = oracle.decode_paged(inp["q"], pg["k_pool"], pg["v_pool"], pg["block_table"], inp["seqlens"], scale)
     assert_close(got, ref, f"{case} splits={num_splits}")
-    # the same arithmetic as the contiguous cache: identical bits
-    assert np.array_equal(got, run_contiguous(gqa, inp, scale, num_splits))
+    # with the same split count, the same arithmetic as the contiguous cache:
+    # identical bits (left to itself the planner gives a paged cache longer
+    # splits, so the automatic counts may differ)
+    if num_splits > 0:
+        assert np.array_equal(got, run_contiguous(gqa, inp, scale, num_splits))
 
 
 @pytest.mark.parametrize("bs", [16, 64])
