@@ -184,6 +184,24 @@ def test_workspace_size_is_zero_for_invalid_shapes(lib):
     assert lib.gqa_decode_workspace_bytes(1, 64, 8, 131072, 128, 0) > 0
 
 
+def test_split_planner_choices(lib):
+    # The automatic split count, seen through the workspace each plan needs
+    # (the partials of nsplit splits): a paged cache gets splits of at least
+    # 448 keys (the Llama-3-8B layer: 19 splits of 448 keys, as asked for
+    # explicitly of the contiguous cache, not the contiguous cache's 26 of
+    # 320), the 8-bit cache about six work items per SM (14 splits), and an
+    # explicit split count gives both layouts the same plan.
+    B, H, K, d, S = 8, 32, 8, 128, 8192
+    contiguous_auto = lib.gqa_decode_workspace_bytes(B, H, K, S, d, 0)
+    assert contiguous_auto == lib.gqa_decode_workspace_bytes(B, H, K, S, d, 26)
+    paged_auto = lib.gqa_decode_paged_workspace_bytes(B, H, K, d, 16, S // 16, 0)
+    assert paged_auto == lib.gqa_decode_workspace_bytes(B, H, K, S, d, 19) < contiguous_auto
+    for ns in (1, 3, 19):
+        assert lib.gqa_decode_paged_workspace_bytes(B, H, K, d, 16, S // 16, ns) == \
+            lib.gqa_decode_workspace_bytes(B, H, K, S, d, ns)
+    assert lib.gqa_decode_int8_workspace_bytes(B, H, K, S, d, 0) == lib.gqa_decode_int8_workspace_bytes(B, H, K, S, d, 14)
+
+
 def _python_imports(path):
     out = set()
     for line in open(path, encoding="utf-8"):
