@@ -52,6 +52,8 @@ SMALL = [
     (4, 1024, 32, 8, 128),  # 512 head-pair units: several per persistent CTA
     (2, 1500, 16, 2, 64),   # G = 8 (four head pairs), d = 64, ragged, several units per CTA
     (1, 700, 16, 4, 128),   # ragged: a last key tile of 60 rows
+    (2, 400, 12, 2, 128),   # G = 6: three head pairs per group
+    (1, 260, 64, 1, 128),   # MQA, G = 64: 32 head pairs share every K/V tile
 ]
 
 

@@ -54,6 +54,8 @@ CASES = [
     ((200, 200, 200), 12, 4, 128),         # equal lengths, G = 3
     (tuple(int(x) for x in np.random.default_rng(5).integers(0, 150, 40)), 4, 2, 64),  # 40 short prompts
     ((900, 1100, 37, 640, 1500), 32, 8, 128),  # 560 head-pair units: several per persistent CTA
+    ((300, 0, 45, 129), 64, 1, 128),       # MQA (G = 64, 32 head pairs) with an empty prompt
+    ((77, 400), 12, 2, 64),                # G = 6, d = 64
 ]
 
 
