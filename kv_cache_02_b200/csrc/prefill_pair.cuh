@@ -634,25 +634,28 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         break;
       }
       tc_fence_after();
-      const int h = g * p.G + 2 * pr + t;
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                            (((size_t)seq0 + qpos) * p.H + h) * D + hh * (D / 2));
-#pragma unroll 1
-      for (int cb = 0; cb < D / 2; cb += 32) {
-        float o[32];
-        tmem_ld32(o_addr + hh * (D / 2) + cb, o);
-        tc_wait_ld();
-        if (qpos < len) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[cb / 8 + i] = make_uint4(pack_bf16x2(o[8 * i] * inv_l, o[8 * i + 1] * inv_l),
-                                         pack_bf16x2(o[8 * i + 2] * inv_l, o[8 * i + 3] * inv_l),
-                                         pack_bf16x2(o[8 * i + 4] * inv_l, o[8 * i + 5] * inv_l),
-                                         pack_bf16x2(o[8 * i + 6] * inv_l, o[8 * i + 7] * inv_l));
-        }
-      }
+      // this half's D / 2 columns of the row, read from TMEM before O_t is released; the
+      // release comes before the global stores (an arrive orders every earlier store of the
+      // thread), so the next unit's first P V does not wait for the output rows to drain:
+      // 0.4915 -> 0.4874 ms on 4 x 4096 x 32 x 128, same box. (Staging the rows through
+      // shared memory so that each store instruction writes whole 128-byte segments, instead
+      // of one 16-byte piece of 32 rows, measured 5 % slower.)
+      float o[D / 2];
+      tmem_ld32(o_addr + hh * (D / 2), *reinterpret_cast<float(*)[32]>(&o[0]));
+      if constexpr (D / 2 > 32) tmem_ld32(o_addr + hh * (D / 2) + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
+      tc_wait_ld();
       tc_fence_before();
       mbar_arrive(&o_free[t]);
+      uint32_t w[D / 4];  // the row's D / 2 outputs, bf16 pairs
+#pragma unroll
+      for (int i = 0; i < D / 4; ++i) w[i] = pack_bf16x2(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
+      const int h = g * p.G + 2 * pr + t;
+      if (qpos < len) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                              (((size_t)seq0 + qpos) * p.H + h) * D + hh * (D / 2));
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
     }
   }
   tc_fence_before();
