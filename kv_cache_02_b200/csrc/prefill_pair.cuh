@@ -650,11 +650,37 @@ __global__ void __launch_bounds__(kPpThreads, 1)
 #pragma unroll
       for (int i = 0; i < D / 4; ++i) w[i] = pack_bf16x2(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
       const int h = g * p.G + 2 * pr + t;
-      if (qpos < len) {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                              (((size_t)seq0 + qpos) * p.H + h) * D + hh * (D / 2));
+      // The row's NC chunks of 16 bytes (chunk c: columns 8 c .. 8 c + 7 of this half) are
+      // transposed across each group of NC lanes by butterfly shuffles, so that store k of
+      // lane j writes chunk j of the group's row k: one store instruction then writes whole
+      // rows of this half (32 / NC rows x D bytes) instead of a 16-byte piece of 32 rows.
+      constexpr int NC = D / 16;
+      const int j = lane & (NC - 1);
 #pragma unroll
-        for (int i = 0; i < D / 16; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      for (int m = 1; m < NC; m <<= 1) {
+        const bool up = (j & m) != 0;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          if (c & m) continue;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t send = up ? w[4 * c + e] : w[4 * (c | m) + e];
+            const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+            if (up)
+              w[4 * c + e] = recv;
+            else
+              w[4 * (c | m) + e] = recv;
+          }
+        }
+      }
+      const int gpos = qt * kPpBM + q * 32 + (lane & ~(NC - 1));  // the group's first query row
+#pragma unroll
+      for (int k = 0; k < NC; ++k) {
+        if (gpos + k < len) {
+          uint4* drow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                 (((size_t)seq0 + gpos + k) * p.H + h) * D + hh * (D / 2));
+          drow[j] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+        }
       }
     }
   }
