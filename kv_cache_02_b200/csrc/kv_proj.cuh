@@ -162,24 +162,64 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       tc_fence_after();
       size_t row = 0;
       const bool valid = m < p.M && (p.splits > 1 || proj_row(p, m, g, row));
+      __syncwarp();  // the lanes reconverge before the warp-collective TMEM loads
+      if (p.splits > 1) {
 #pragma unroll 1
-      for (int cb = 0; cb < C::kN; cb += 32) {
-        float o[32];
-        tmem_ld32(lane_addr + cb, o);  // warp-collective: every lane takes part
-        tc_wait_ld();
-        if (!valid) continue;
-        if (p.splits > 1) {
-          float4* dst = reinterpret_cast<float4*>(p.ws + ((size_t)sp * p.M + m) * ((size_t)p.K * C::kN) +
-                                                  (size_t)g * C::kN + cb);
+        for (int cb = 0; cb < C::kN; cb += 32) {
+          float o[32];
+          tmem_ld32(lane_addr + cb, o);  // warp-collective: every lane takes part
+          tc_wait_ld();
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(p.ws + ((size_t)sp * p.M + m) * ((size_t)p.K * C::kN) +
+                                                    (size_t)g * C::kN + cb);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-        } else {
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
+          __syncwarp();  // converged again for the next TMEM loads
+        }
+      } else {
+        // 64 columns (a 128-byte segment of a cache row) at a time. Thread r holds token r's
+        // row, so a store instruction would write a 16-byte piece of 32 rows; the 8 pieces are
+        // transposed across each group of 8 lanes by butterfly shuffles, and store k of lane j
+        // writes piece j of the group's row k: 4 whole segments per instruction.
+        const int j = lane & 7;
+#pragma unroll 1
+        for (int cb = 0; cb < C::kN; cb += 64) {
+          float o[64];
+          tmem_ld32(lane_addr + cb, *reinterpret_cast<float(*)[32]>(&o[0]));
+          tmem_ld32(lane_addr + cb + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
+          tc_wait_ld();
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
+#pragma unroll
+          for (int mk = 1; mk < 8; mk <<= 1) {
+            const bool up = (j & mk) != 0;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              if (c & mk) continue;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint32_t send = up ? w[4 * c + e] : w[4 * (c | mk) + e];
+                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, mk);
+                if (up)
+                  w[4 * c + e] = recv;
+                else
+                  w[4 * (c | mk) + e] = recv;
+              }
+            }
+          }
           __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(cb < D ? p.k_cache : p.v_cache);
-          uint4* dst = reinterpret_cast<uint4*>(cache + row * D + (cb % D));
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pack_bf16x2(o[8 * i], o[8 * i + 1]), pack_bf16x2(o[8 * i + 2], o[8 * i + 3]),
-                                pack_bf16x2(o[8 * i + 4], o[8 * i + 5]), pack_bf16x2(o[8 * i + 6], o[8 * i + 7]));
+          for (int k = 0; k < 8; ++k) {
+            const int src = (lane & ~7) + k;  // the lane that holds row k of the group
+            const unsigned long long rk = __shfl_sync(0xffffffffu, (unsigned long long)row, src);
+            const bool vk = __shfl_sync(0xffffffffu, valid ? 1 : 0, src) != 0;
+            if (vk)
+              reinterpret_cast<uint4*>(cache + rk * D + (cb % D))[j] =
+                  make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          }
+          __syncwarp();  // converged again for the next TMEM loads
         }
       }
     }

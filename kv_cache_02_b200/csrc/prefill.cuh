@@ -409,20 +409,44 @@ __global__ void __launch_bounds__(kPfThreads, 2)
       tc_fence_after();
       const float inv_l = 1.f / l;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-      uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)seq0 + qpos) * p.H + h) * D);
+      // 64 columns at a time; the row's eight 16-byte pieces are transposed across each group
+      // of 8 lanes (butterfly shuffles) so that each store instruction writes 4 rows x 128
+      // contiguous bytes instead of a 16-byte piece of 32 rows
+      const int j = lane & 7;
 #pragma unroll 1
-      for (int cb = 0; cb < D; cb += 32) {
-        float o[32];
-        tmem_ld32(lane_addr + C::kOCol + cb, o);
+      for (int cb = 0; cb < D; cb += 64) {
+        float o[64];
+        tmem_ld32(lane_addr + C::kOCol + cb, *reinterpret_cast<float(*)[32]>(&o[0]));
+        tmem_ld32(lane_addr + C::kOCol + cb + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
         tc_wait_ld();
-        if (qpos < len) {
+        uint32_t w[32];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[cb / 8 + i] = make_uint4(pack_bf16x2(o[8 * i] * inv_l, o[8 * i + 1] * inv_l),
-                                         pack_bf16x2(o[8 * i + 2] * inv_l, o[8 * i + 3] * inv_l),
-                                         pack_bf16x2(o[8 * i + 4] * inv_l, o[8 * i + 5] * inv_l),
-                                         pack_bf16x2(o[8 * i + 6] * inv_l, o[8 * i + 7] * inv_l));
+        for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
+#pragma unroll
+        for (int mk = 1; mk < 8; mk <<= 1) {
+          const bool up = (j & mk) != 0;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (c & mk) continue;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t send = up ? w[4 * c + e] : w[4 * (c | mk) + e];
+              const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, mk);
+              if (up)
+                w[4 * c + e] = recv;
+              else
+                w[4 * (c | mk) + e] = recv;
+            }
+          }
         }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int qk = __shfl_sync(0xffffffffu, qpos, (lane & ~7) + k);  // row k of the group
+          if (qk < len)
+            reinterpret_cast<uint4*>(out + (((size_t)seq0 + qk) * p.H + h) * D + cb)[j] =
+                make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+        }
+        __syncwarp();  // converged again for the next warp-collective TMEM loads
       }
     }
   }

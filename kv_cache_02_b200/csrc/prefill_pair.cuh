@@ -682,6 +682,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
           drow[j] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
         }
       }
+      __syncwarp();  // converged again before the next unit's warp-collective TMEM loads
     }
   }
   tc_fence_before();
