@@ -56,6 +56,10 @@ CASES = [
     ((900, 1100, 37, 640, 1500), 32, 8, 128),  # 560 head-pair units: several per persistent CTA
     ((300, 0, 45, 129), 64, 1, 128),       # MQA (G = 64, 32 head pairs) with an empty prompt
     ((77, 400), 12, 2, 64),                # G = 6, d = 64
+    (tuple(int(x) for x in np.random.default_rng(9).integers(0, 300, 256)), 8, 2, 64),  # 256 prompts: the
+    # most that the per-CTA unit list takes, 1 to 3 query tiles each
+    (tuple(int(x) for x in np.random.default_rng(11).integers(0, 60, 300)), 4, 2, 64),  # 300 prompts: the
+    # sequence-major order
 ]
 
 
